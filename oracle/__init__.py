@@ -1,0 +1,204 @@
+"""CPU oracle for the MoE token round trip (route, dispatch, SwiGLU FFN, combine).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline / reference leg of ``bench.py``.  The product library
+(``token_dispatch_combine_b200``) never imports it, and the two share no code.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, float64); this module only
+builds it with gcc and marshals numpy arrays.  Each C function cites the page
+passage it follows.  Every function is pinned by ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F32, BF16 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into liboracle.so (gcc -O2, OpenMP, strict IEEE)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _configure(lib):
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.oracle_route.argtypes = [vp, i32, i32, i32, vp, vp]
+    lib.oracle_route.restype = i32
+    lib.oracle_src_rank.argtypes = [i32, i32, i32]
+    lib.oracle_src_rank.restype = i32
+    lib.oracle_dispatch_index.argtypes = [vp, i32, i32, i32, i32] + [vp] * 7
+    lib.oracle_dispatch_index.restype = i32
+    lib.oracle_dispatch_rows.argtypes = [vp, sz, i32, i32, vp, vp]
+    lib.oracle_ffn_rows.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, i32, i32, vp, vp]
+    lib.oracle_combine.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+    return lib
+
+
+def _get():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _configure(ctypes.CDLL(build()))
+    return _lib
+
+
+@contextlib.contextmanager
+def _substitute_library(path: str):
+    """Run the wrappers against another build of the oracle source (used by the
+    mutation tests, which plant a mistake in a copy and expect a pin to fail)."""
+    global _lib
+    _get()
+    saved = _lib
+    _lib = _configure(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def route(logits: np.ndarray, k: int):
+    """Top-k ids [T,k] int32 (logit desc, lower id on ties) and softmax weights [T,k] float32."""
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    if _get().oracle_route(logits.ctypes.data, T, E, k, ids.ctypes.data, w.ctypes.data) != 0:
+        raise ValueError("oracle_route: bad sizes")
+    return ids, w
+
+
+def src_rank(t: int, T: int, R: int) -> int:
+    return _get().oracle_src_rank(t, T, R)
+
+
+def dispatch_index(ids: np.ndarray, E: int, R: int) -> dict:
+    """Counts, offsets and the stable slot<->row permutation (see moe_oracle.c)."""
+    ids = _c(ids, np.int32)
+    T, k = ids.shape
+    S = T * k
+    out = dict(
+        expert_counts=np.empty(E, np.int32), expert_offsets=np.empty(E + 1, np.int32),
+        rank_counts=np.empty(R, np.int32), rank_offsets=np.empty(R + 1, np.int32),
+        slot_to_row=np.empty(S, np.int32), row_to_slot=np.empty(S, np.int32),
+        src_expert_counts=np.empty((R, E), np.int32),
+    )
+    dropped = _get().oracle_dispatch_index(
+        ids.ctypes.data, T, k, E, R, *(out[n].ctypes.data for n in (
+            "expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "slot_to_row",
+            "row_to_slot", "src_expert_counts")))
+    if dropped < 0:
+        raise ValueError("oracle_dispatch_index: bad sizes")
+    out["dropped"] = dropped
+    return out
+
+
+def dispatch_rows(x: np.ndarray, k: int, slot_to_row: np.ndarray, n_rows: int | None = None) -> np.ndarray:
+    """x_disp[slot_to_row[s]] = x[s // k]; rows never written stay zero."""
+    x = np.ascontiguousarray(x)
+    T = x.shape[0]
+    n_rows = T * k if n_rows is None else n_rows
+    xd = np.zeros((n_rows,) + x.shape[1:], dtype=x.dtype)
+    s2r = _c(slot_to_row, np.int32)
+    _get().oracle_dispatch_rows(x.ctypes.data, x[0].nbytes if T else 0, T, k, s2r.ctypes.data, xd.ctypes.data)
+    return xd
+
+
+def _dt(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    raise TypeError(f"oracle takes float32 or bfloat16 bits (uint16), got {a.dtype}")
+
+
+def ffn_rows(x_rows: np.ndarray, row_expert: np.ndarray, w_gate, w_up, w_down, H: int, I: int,
+             want_act: bool = False):
+    """SwiGLU expert MLP of each row in float64.
+
+    ``w_gate``/``w_up``/``w_down`` map expert id -> that expert's matrix
+    ([H,I], [H,I], [I,H]; float32 or bf16 bits).  They may be full [E,...]
+    arrays or dicts holding only the experts that ``row_expert`` uses.
+    Returns y [n,H] (and the activations [n,I] when ``want_act``).
+    """
+    x_rows = np.ascontiguousarray(x_rows)
+    n = x_rows.shape[0]
+    rexp = _c(row_expert, np.int32)
+    if isinstance(w_gate, np.ndarray):
+        E = w_gate.shape[0]
+        g = {e: w_gate[e] for e in range(E)}
+        u = {e: w_up[e] for e in range(E)}
+        d = {e: w_down[e] for e in range(E)}
+    else:
+        g, u, d = w_gate, w_up, w_down
+    E = (max(g.keys()) + 1) if g else 1
+    keep = []
+
+    def ptrs(m):
+        arr = (ctypes.c_void_p * E)()
+        for e, a in m.items():
+            a = np.ascontiguousarray(a)
+            keep.append(a)
+            arr[e] = a.ctypes.data
+        return arr
+
+    pg, pu, pd = ptrs(g), ptrs(u), ptrs(d)
+    wdt = _dt(next(iter(g.values()))) if g else F32
+    for e in set(rexp.tolist()):
+        if e not in g:
+            raise KeyError(f"weights of expert {e} not supplied")
+    y = np.empty((n, H), np.float64)
+    a = np.empty((n, I), np.float64) if want_act else None
+    if n:
+        _get().oracle_ffn_rows(x_rows.ctypes.data, _dt(x_rows), rexp.ctypes.data, n, pg, pu, pd, wdt, H, I,
+                               a.ctypes.data if want_act else None, y.ctypes.data)
+    return (y, a) if want_act else y
+
+
+def combine(y_disp: np.ndarray, topk_w: np.ndarray, slot_to_row: np.ndarray) -> np.ndarray:
+    """y[t] = sum_j w[t,j] * y_disp[slot_to_row[t*k+j]] in float64."""
+    y_disp = _c(y_disp, np.float64)
+    topk_w = _c(topk_w, np.float32)
+    s2r = _c(slot_to_row, np.int32)
+    T, k = topk_w.shape
+    H = y_disp.shape[1]
+    y = np.empty((T, H), np.float64)
+    _get().oracle_combine(y_disp.ctypes.data, topk_w.ctypes.data, s2r.ctypes.data, T, k, H, y.ctypes.data)
+    return y
+
+
+def round_trip(x: np.ndarray, logits: np.ndarray, k: int, E: int, R: int, w_gate, w_up, w_down):
+    """The whole layer on the CPU: route -> dispatch -> FFN -> combine.  Returns a dict of every stage."""
+    H = x.shape[1]
+    I = w_gate.shape[-1] if isinstance(w_gate, np.ndarray) else next(iter(w_gate.values())).shape[-1]
+    ids, w = route(logits, k)
+    idx = dispatch_index(ids, E, R)
+    x_disp = dispatch_rows(x, k, idx["slot_to_row"])
+    S = ids.size
+    row_expert = np.repeat(np.arange(E, dtype=np.int32), idx["expert_counts"])
+    n = int(idx["expert_offsets"][-1])
+    y_disp, act = ffn_rows(x_disp[:n], row_expert, w_gate, w_up, w_down, H, I, want_act=True)
+    if n < S:
+        y_disp = np.concatenate([y_disp, np.zeros((S - n, H))])
+    y = combine(y_disp, w, idx["slot_to_row"])
+    return dict(ids=ids, w=w, x_disp=x_disp, act=act, y_disp=y_disp, y=y, **idx)

@@ -1,0 +1,234 @@
+/*
+ * CPU oracle for the MoE expert-parallel token round trip.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  The product path
+ * (the CUDA library) never calls it and shares no code with it.
+ *
+ * It computes, slowly and directly, what the round trip computes:
+ *   route    -> top-k expert ids per token + softmax over the k chosen logits
+ *   index    -> per-expert counts, exclusive offsets, per-rank counts and
+ *               offsets, per-(source rank, expert) counts, and the stable
+ *               slot <-> row permutation
+ *   dispatch -> copy of each token row to every row it was dispatched to
+ *   ffn      -> per-row SwiGLU expert MLP, in float64
+ *   combine  -> weighted sum of a token's k expert outputs, in float64
+ *
+ * Floating point is float64 throughout (inputs are widened exactly); the
+ * pages fix no precision.  Notation: T tokens, H hidden, I intermediate,
+ * E experts, k experts per token, R logical EP ranks, S = T*k slots; slot
+ * s = t*k + j is the j-th choice of token t.
+ *
+ * Sources (page title, section):
+ *  [EPRT]  "EP: Partition Experts and Route Tokens" -- sections "Send tokens
+ *          to experts and return their results", "Return multiple expert
+ *          results to the same token", "Equal expert counts can receive
+ *          different token counts".
+ *  [NEURON] "Expert Parallelism (EP)" (vLLM on Neuron design note) --
+ *          sections "Weight Layout Across Ranks", "Collective Patterns /
+ *          Prefill (CTE kernel)", "Why a Single All-Reduce/Reduce-Scatter
+ *          Works", "Limitations" (items 1, 3 and 4).
+ *  [SWIGLU] Shazeer, "GLU Variants Improve Transformer" (2020): FFN_SwiGLU(x)
+ *          = (SiLU(x W) * (x V)) W2, SiLU(z) = z * sigmoid(z).  The pages call
+ *          each expert "an MLP"; the layer shapes name its form SwiGLU.
+ *
+ * Parity pins: every function here is checked by the not-gpu tests against
+ * the pages' worked examples, closed forms and a dense brute-force MoE.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_F32 0
+#define ORC_BF16 1
+
+static double orc_load(const void* base, int dtype, size_t i) {
+  if (dtype == ORC_F32) return (double)((const float*)base)[i];
+  uint32_t u = (uint32_t)((const uint16_t*)base)[i] << 16; /* exact widening */
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* ------------------------------------------------------------------ route
+ * [EPRT] "Send tokens ...": the router chooses each token's expert(s) from
+ * all E experts; Top-1 uses combination weight one.  "Return multiple ...":
+ * with Top-2 the token's results are combined with per-expert weights kept
+ * apart from the expert choice.  Weight rule: softmax over the k selected
+ * logits (which gives exactly 1 for k = 1).
+ *
+ * Order: experts sorted by logit descending; equal logits (IEEE ==, so
+ * -0 == +0) keep the lower expert id first.  Plain repeated selection.
+ * Returns 0, or -1 for bad sizes.
+ */
+int oracle_route(const float* logits, int T, int E, int k, int32_t* ids, float* w) {
+  if (T < 0 || E < 1 || k < 1 || k > E || k > 64) return -1;
+  unsigned char* taken = (unsigned char*)malloc((size_t)E);
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + (size_t)t * E;
+    memset(taken, 0, (size_t)E);
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        if (best < 0 || l[e] > l[best]) best = e; /* strict: ties keep lower id */
+      }
+      taken[best] = 1;
+      ids[(size_t)t * k + j] = best;
+    }
+    double m = (double)l[ids[(size_t)t * k]];
+    double z = 0.0;
+    double ex[64];
+    for (int j = 0; j < k && j < 64; ++j) {
+      ex[j] = exp((double)l[ids[(size_t)t * k + j]] - m);
+      z += ex[j];
+    }
+    for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = (float)(ex[j] / z);
+  }
+  free(taken);
+  return 0;
+}
+
+/* Source rank of token t when T tokens are split into R contiguous, as-equal-
+ * as-possible ranges (t in [ceil(rT/R), ceil((r+1)T/R)) belongs to rank r).
+ * With R | T this is t / (T/R): tokens 0..T/R-1 on rank 0, and so on, as in
+ * [EPRT] "Replicate attention ...": each GPU holds its own tokens. */
+int oracle_src_rank(int t, int T, int R) { return (int)(((int64_t)t * R) / T); }
+
+/* ------------------------------------------------------------------ index
+ * [EPRT] "Send tokens ...": dispatch groups token vectors by the selected
+ * expert and keeps each result's association to its original token;
+ * "Equal expert counts ...": experts and ranks receive unequal counts.
+ * [NEURON] "Limitations" 3-4: rank r owns experts [r*E/R, (r+1)*E/R).
+ *
+ * Rows are ordered by (expert, token): expert e's rows start at the
+ * exclusive prefix sum of the counts of experts < e, and within an expert
+ * the rows follow token order (a stable grouping).  Because experts are
+ * placed contiguously, that order is also rank-major.
+ *
+ * Slots whose id is outside [0, E) are dropped: not counted, slot_to_row
+ * = -1.  row_to_slot entries past the last placed row are -1.
+ * src_expert_counts may be NULL.  Returns the number of dropped slots, or
+ * -1 for bad sizes.
+ */
+int oracle_dispatch_index(const int32_t* ids, int T, int k, int E, int R,
+                          int32_t* expert_counts, int32_t* expert_offsets,
+                          int32_t* rank_counts, int32_t* rank_offsets,
+                          int32_t* slot_to_row, int32_t* row_to_slot,
+                          int32_t* src_expert_counts) {
+  if (T < 0 || k < 1 || E < 1 || R < 1 || E % R != 0) return -1;
+  const int S = T * k, EL = E / R;
+  int dropped = 0;
+  for (int e = 0; e < E; ++e) expert_counts[e] = 0;
+  for (int s = 0; s < S; ++s) {
+    if (ids[s] < 0 || ids[s] >= E) { ++dropped; continue; }
+    expert_counts[ids[s]] += 1;
+  }
+  expert_offsets[0] = 0;
+  for (int e = 0; e < E; ++e) expert_offsets[e + 1] = expert_offsets[e] + expert_counts[e];
+  for (int r = 0; r < R; ++r) {
+    rank_counts[r] = 0;
+    for (int e = r * EL; e < (r + 1) * EL; ++e) rank_counts[r] += expert_counts[e];
+  }
+  rank_offsets[0] = 0;
+  for (int r = 0; r < R; ++r) rank_offsets[r + 1] = rank_offsets[r] + rank_counts[r];
+
+  int32_t* cursor = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+  for (int s = 0; s < S; ++s) row_to_slot[s] = -1;
+  for (int t = 0; t < T; ++t) {
+    for (int j = 0; j < k; ++j) {
+      int s = t * k + j, e = ids[s];
+      if (e < 0 || e >= E) { slot_to_row[s] = -1; continue; }
+      int row = expert_offsets[e] + cursor[e]++;
+      slot_to_row[s] = row;
+      row_to_slot[row] = s;
+    }
+  }
+  free(cursor);
+  if (src_expert_counts) {
+    memset(src_expert_counts, 0, sizeof(int32_t) * (size_t)R * E);
+    for (int s = 0; s < S; ++s) {
+      int e = ids[s];
+      if (e < 0 || e >= E) continue;
+      src_expert_counts[(size_t)oracle_src_rank(s / k, T, R) * E + e] += 1;
+    }
+  }
+  return dropped;
+}
+
+/* ---------------------------------------------------------------- dispatch
+ * [EPRT] "Send tokens ...": experts receive the token input vectors (not the
+ * router scores).  x_disp[slot_to_row[s]] = x[s / k], a byte copy. */
+void oracle_dispatch_rows(const void* x, size_t row_bytes, int T, int k,
+                          const int32_t* slot_to_row, void* x_disp) {
+  for (int s = 0; s < T * k; ++s) {
+    if (slot_to_row[s] < 0) continue;
+    memcpy((char*)x_disp + (size_t)slot_to_row[s] * row_bytes,
+           (const char*)x + (size_t)(s / k) * row_bytes, row_bytes);
+  }
+}
+
+/* --------------------------------------------------------------------- ffn
+ * [EPRT] "Send tokens ...": an expert transforms each of its rows on its
+ * own (rows are stacked only to batch the work).  [SWIGLU]:
+ *   g = x . Wg_e,  u = x . Wu_e          (Wg_e, Wu_e: [H, I], row-major)
+ *   a = SiLU(g) * u,  SiLU(z) = z / (1 + exp(-z))
+ *   y = a . Wd_e                          (Wd_e: [I, H], row-major)
+ * All sums in float64, ascending index.
+ *
+ * Computes n rows: row i has input x_rows[i*H ..] (dtype xdt), expert
+ * row_expert[i]; w_gate[e], w_up[e], w_down[e] point at expert e's matrices
+ * (dtype wdt; entries of unused experts may be NULL).  a_out (n x I, may be
+ * NULL) receives the SwiGLU activations, y_out (n x H) the outputs.
+ */
+void oracle_ffn_rows(const void* x_rows, int xdt, const int32_t* row_expert, int n,
+                     const void* const* w_gate, const void* const* w_up,
+                     const void* const* w_down, int wdt, int H, int I,
+                     double* a_out, double* y_out) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < n; ++i) {
+    int e = row_expert[i];
+    double* x = (double*)malloc(sizeof(double) * (size_t)H);
+    double* g = (double*)calloc((size_t)I, sizeof(double));
+    double* u = (double*)calloc((size_t)I, sizeof(double));
+    double* y = y_out + (size_t)i * H;
+    for (int h = 0; h < H; ++h) x[h] = orc_load(x_rows, xdt, (size_t)i * H + h);
+    for (int h = 0; h < H; ++h) {
+      for (int c = 0; c < I; ++c) {
+        g[c] += x[h] * orc_load(w_gate[e], wdt, (size_t)h * I + c);
+        u[c] += x[h] * orc_load(w_up[e], wdt, (size_t)h * I + c);
+      }
+    }
+    for (int c = 0; c < I; ++c) {
+      g[c] = g[c] / (1.0 + exp(-g[c])) * u[c];
+      if (a_out) a_out[(size_t)i * I + c] = g[c];
+    }
+    for (int h = 0; h < H; ++h) y[h] = 0.0;
+    for (int c = 0; c < I; ++c)
+      for (int h = 0; h < H; ++h) y[h] += g[c] * orc_load(w_down[e], wdt, (size_t)c * H + h);
+    free(x);
+    free(g);
+    free(u);
+  }
+}
+
+/* ----------------------------------------------------------------- combine
+ * [EPRT] "Send tokens ...": results return to their original tokens and
+ * original order; "Return multiple ...": y(t) = sum_j w[t,j] * u_j, e.g.
+ * y(A2) = 0.7 u0 + 0.3 u2.  Sum in float64 over j ascending.
+ * y_disp holds float64 expert outputs indexed by row; slots with
+ * slot_to_row < 0 contribute nothing. */
+void oracle_combine(const double* y_disp, const float* topk_w, const int32_t* slot_to_row,
+                    int T, int k, int H, double* y) {
+  for (int t = 0; t < T; ++t) {
+    double* out = y + (size_t)t * H;
+    for (int h = 0; h < H; ++h) out[h] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      int row = slot_to_row[(size_t)t * k + j];
+      if (row < 0) continue;
+      double wj = (double)topk_w[(size_t)t * k + j];
+      for (int h = 0; h < H; ++h) out[h] += wj * y_disp[(size_t)row * H + h];
+    }
+  }
+}

@@ -1,0 +1,67 @@
+"""Plant one mistake at a time in a copy of the oracle source (on the CPU) and
+check that at least one pin in test_oracle_pins fails for each.  Every planted
+mistake keeps all memory accesses in bounds."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
+
+MUTANTS = {
+    "tie_keeps_higher_id": ("l[e] > l[best]", "l[e] >= l[best]"),
+    "softmax_not_normalised": ("(float)(ex[j] / z)", "(float)(ex[j])"),
+    "gate_and_up_swapped": ("g[c] = g[c] / (1.0 + exp(-g[c])) * u[c];", "g[c] = u[c] / (1.0 + exp(-u[c])) * g[c];"),
+    "down_weight_transposed": ("(size_t)c * H + h", "(size_t)h * I + c"),
+    "gate_weight_transposed": ("orc_load(w_gate[e], wdt, (size_t)h * I + c)", "orc_load(w_gate[e], wdt, (size_t)c * H + h)"),
+    "rows_in_reverse_token_order": ("for (int t = 0; t < T; ++t) {\n    for (int j = 0; j < k; ++j) {\n      int s = t * k + j, e = ids[s];",
+                                    "for (int t = T - 1; t >= 0; --t) {\n    for (int j = 0; j < k; ++j) {\n      int s = t * k + j, e = ids[s];"),
+    "offsets_not_accumulated": ("expert_offsets[e + 1] = expert_offsets[e] + expert_counts[e];",
+                                "expert_offsets[e + 1] = expert_counts[e];"),
+    "rank_offsets_not_accumulated": ("rank_offsets[r + 1] = rank_offsets[r] + rank_counts[r];",
+                                     "rank_offsets[r + 1] = rank_counts[r];"),
+    "round_robin_placement": ("for (int e = r * EL; e < (r + 1) * EL; ++e)", "for (int e = r; e < E; e += R)"),
+    "src_rank_round_robin": ("(int)(((int64_t)t * R) / T)", "(t % R)"),
+    "combine_ignores_weight": ("out[h] += wj * y_disp", "out[h] += y_disp"),
+    "combine_drops_last_choice": ("for (int j = 0; j < k; ++j) {\n      int row = slot_to_row", "for (int j = 0; j < k - 1; ++j) {\n      int row = slot_to_row"),
+}
+
+PINS = [
+    pins.test_worked_example_route_and_dispatch,
+    pins.test_worked_example_results_return_in_original_order,
+    pins.test_top2_weights_and_combine,
+    pins.test_imbalance_example,
+    pins.test_masked_sum_ep8,
+    pins.test_route_ties_lower_id_first_and_signed_zero,
+    lambda: pins.test_route_matches_lexsort(37, 8, 2),
+    lambda: pins.test_dispatch_index_invariants(127, 8, 2, 4),
+    pins.test_src_rank_matches_toy_layer_statement,
+    pins.test_swiglu_closed_forms,
+    lambda: pins.test_round_trip_equals_dense_masked_moe(16, 32, 64, 8, 2, 4),
+    pins.test_identity_experts_reproduce_input,
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc missing")
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path = tmp_path / "mut.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(so), str(path), "-lm"])
+    caught = []
+    with oracle._substitute_library(str(so)):
+        for pin in PINS:
+            try:
+                pin()
+            except Exception:  # a failed assertion, or a wrong value that breaks the check itself
+                caught.append(getattr(pin, "__name__", "pin"))
+    assert caught, f"mutant {name} passed every pin"
