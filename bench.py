@@ -1,0 +1,396 @@
+"""Benchmark of the MoE expert-parallel token round trip on B200.
+
+One step = one pass of the whole round trip over one batch: route ->
+dispatch -> grouped SwiGLU FFN (gate/up, down) -> combine, through the C ABI.
+Default workload: the GPT-OSS-20B-shaped layer with balanced routing
+(T=4096, H=2880, I=3072, E=32, top-4, R=8 logical ranks, bf16).
+
+Prints ONE JSON line on rank 0.  Under torchrun each GPU runs its own
+independent copy of the layer on its own batch (weak scaling, no data-path
+collective); time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; dispatch+combine HBM GB/s; grouped-GEMM TFLOP/s vs peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20  # > 126 MB of L2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("ffn_tc.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "token_dispatch_combine_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(workload: str):
+    """Per-launch DRAM bytes of the gate/up kernel from the committed ncu summary,
+    if it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload and parts[1] == "gate_up" \
+                and parts[3] == sha:
+            return int(float(parts[2]))
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML during the timed region."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        n = self.nvml
+        self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+        mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for name, bit in self.REASONS.items():
+            if mask & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nvml:
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nvml:
+            self.t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(values, world):
+    import torch
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def algorithmic(wl):
+    b = 2 if wl.dtype == "bf16" else 4
+    S = wl.S
+    return {
+        "dispatch_bytes": wl.T * wl.H * b + S * wl.H * b + 12 * S,  # x read, x_disp write, ids/ranks/maps
+        "combine_bytes": S * wl.H * b + wl.T * wl.H * b + 8 * S,  # y_disp read, y write, w + slot_to_row
+        "route_bytes": wl.T * wl.E * 4 + wl.T * wl.k * 8,
+        "gateup_flops": 4.0 * S * wl.H * wl.I,
+        "down_flops": 2.0 * S * wl.H * wl.I,
+    }
+
+
+# --------------------------------------------------------------------------- CPU oracle legs
+def oracle_sample_step(wl, x, logits, wg, wu, wd, n_tok, rng):
+    """The oracle's round trip on a batch of n_tok tokens of the workload."""
+    import oracle
+    idx = np.sort(rng.choice(wl.T, size=n_tok, replace=False))
+    t0 = time.perf_counter()
+    oracle.round_trip(x[idx], logits[idx], wl.k, wl.E, wl.R, wg, wu, wd)
+    return time.perf_counter() - t0
+
+
+def size_oracle_sample(wl, x, logits, wg, wu, wd, target_s, rng):
+    n = max(1, min(wl.T, 4))
+    dt = oracle_sample_step(wl, x, logits, wg, wu, wd, n, rng)
+    per_tok = dt / n
+    return int(max(1, min(wl.T, target_s / max(per_tok, 1e-9)))), per_tok
+
+
+def cpu_cores():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def host_inputs(wl):
+    x = wl.x()
+    logits = wl.logits(synth.bf16_bits_to_f32(x) if wl.dtype == "bf16" else x)
+    return x, logits, wl.w_gate(), wl.w_up(), wl.w_down()
+
+
+def run_reference(args, wl):
+    """Reference arm: the CPU oracle, timed on the host cores, rank 0 only."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x, logits, wg, wu, wd = host_inputs(wl)
+    rng = np.random.default_rng(0)
+    n_tok, _ = size_oracle_sample(wl, x, logits, wg, wu, wd, target_s=2.0, rng=rng)
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, x, logits, wg, wu, wd, n_tok, rng)
+    times = [oracle_sample_step(wl, x, logits, wg, wu, wd, n_tok, rng) for _ in range(args.steps)]
+    total = sum(times)
+    value = n_tok * args.steps / total
+    sample = f"{n_tok} of {wl.T} tokens per step (whole round trip on that batch, same layer)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(wl):
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "R": wl.R,
+            "dtype": wl.dtype, "routing_bias": wl.bias, "seed": wl.seed,
+            "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)"}
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, wl):
+    import torch
+
+    from token_dispatch_combine_b200 import MoERoundTrip, moe_get_error
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+    x_np, logits_np, wg_np, wu_np, wd_np = host_inputs(wl)
+
+    def up(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.to(dev).view(dt) if a.dtype == np.uint16 else t.to(dev)
+
+    x, logits = up(x_np), up(logits_np)
+    wg, wu, wd = up(wg_np), up(wu_np), up(wd_np)
+    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev):
+        ev[0].record(stream)
+        rt.route(logits)
+        ev[1].record(stream)
+        rt.dispatch(x)
+        ev[2].record(stream)
+        rt.gate_up(wg, wu)
+        ev[3].record(stream)
+        rt.down(wd)
+        ev[4].record(stream)
+        rt.combine()
+        ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(6)])
+    st, bits = moe_get_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {bits} during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()  # outside the timed events: inputs start cold in L2
+            step(events[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    stage = np.zeros(5)
+    for ev in events:
+        stage += [ev[j].elapsed_time(ev[j + 1]) for j in range(5)]
+    stage /= args.steps  # ms per step per stage: route, dispatch, gate_up, down, combine
+    step_ms = float(stage.sum())
+    step_ms, *stage_max = max_over_ranks([step_ms, *stage.tolist()], world)
+
+    # end to end through the public API, host buffers (pinned), copies inside the timed region
+    x_h = torch.from_numpy(x_np.view(np.int16) if x_np.dtype == np.uint16 else x_np).pin_memory()
+    l_h = torch.from_numpy(logits_np).pin_memory()
+    y_h = torch.empty((wl.T, wl.H), dtype=torch.int16 if dt == torch.bfloat16 else torch.float32).pin_memory()
+    x_d = torch.empty_like(x)
+    l_d = torch.empty_like(logits)
+
+    def e2e_step():
+        x_d.view(x_h.dtype).copy_(x_h, non_blocking=True)
+        l_d.copy_(l_h, non_blocking=True)
+        y = rt.forward(x_d, l_d, wg, wu, wd)
+        y_h.copy_(y.view(y_h.dtype), non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        flush.zero_()
+        e2e_step()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for a, b in e2e_ev:
+        flush.zero_()
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+    (e2e_ms,) = max_over_ranks([e2e_ms], world)
+    st, bits = moe_get_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {bits} during timing")
+
+    if rank != 0:
+        return 0
+    peaks, peak_src = load_peaks()
+    alg = algorithmic(wl)
+    t_route, t_disp, t_gu, t_down, t_comb = stage_max
+    gemm_tflops = (alg["gateup_flops"] + alg["down_flops"]) / ((t_gu + t_down) * 1e-3) / 1e12
+    dc_gbs = (alg["dispatch_bytes"] + alg["combine_bytes"]) / ((t_disp + t_comb) * 1e-3) / 1e9
+    gu_tflops = alg["gateup_flops"] / (t_gu * 1e-3) / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    cpu = None
+    if args.cpu_baseline and world == 1:
+        rng = np.random.default_rng(1)
+        n_tok, _ = size_oracle_sample(wl, x_np, logits_np, wg_np, wu_np, wd_np, target_s=12.0, rng=rng)
+        secs = oracle_sample_step(wl, x_np, logits_np, wg_np, wu_np, wd_np, n_tok, rng)
+        cpu = {"value": n_tok / secs, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"{n_tok} of {wl.T} tokens through the whole round trip ({secs:.1f} s)"}
+    line = {
+        "metric": METRIC,
+        "value": wl.T * world / (step_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": config_dict(wl),
+        "components": {
+            "route_us": t_route * 1e3, "dispatch_us": t_disp * 1e3, "gate_up_us": t_gu * 1e3,
+            "down_us": t_down * 1e3, "combine_us": t_comb * 1e3,
+            "dispatch_combine_gbs": dc_gbs, "dispatch_combine_frac_hbm": dc_gbs / peaks["hbm_gbs"],
+            "grouped_gemm_tflops": gemm_tflops, "grouped_gemm_frac_bf16": gemm_tflops / peak_tf,
+        },
+        "roofline": {
+            "kernel": "grouped_gemm_tc_kernel<gate/up, SwiGLU epilogue>",
+            "bound": "tensor", "achieved": gu_tflops, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": gu_tflops / peak_tf, "traffic": dram_traffic(wl.name),
+            "peak_source": f"{peak_src} bf16 dense (burst)",
+            "algorithmic_per_launch": f"4*S*H*I = {alg['gateup_flops']:.4g} FLOP",
+        },
+        "e2e": {"value": wl.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_np.nbytes + logits_np.nbytes), "d2h_bytes_per_step": int(x_np.nbytes)},
+        "gpu_launches": MoERoundTrip.KERNELS_PER_FORWARD * args.steps,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="gptoss_uniform", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false",
+                    help="skip the CPU oracle leg (used for profiler runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = synth.WORKLOADS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    rc = run_ours(args, wl)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,198 @@
+/*
+ * moe_b200.h -- C ABI of the MoE expert-parallel token round trip on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * One MoE layer's token round trip, as four calls:
+ *
+ *   moe_route      logits -> top-k expert ids + softmax-over-top-k weights
+ *   moe_dispatch   expert histogram, exclusive scan, stable scatter of token
+ *                  rows into an expert-contiguous (= rank-major) buffer,
+ *                  per-expert / per-rank / per-(source rank, expert) counts
+ *   moe_expert_ffn grouped SwiGLU expert MLP over the ragged expert segments
+ *                  (also callable as its two halves, moe_ffn_gate_up and
+ *                  moe_ffn_down)
+ *   moe_combine    gather each token's k expert outputs, weight them by the
+ *                  router weights, sum, and write them in original token order
+ *
+ * Sources (page title, section):
+ *  [EPRT]   "EP: Partition Experts and Route Tokens": "Send tokens to experts
+ *           and return their results" (route, dispatch, per-expert batched
+ *           MLP, return in original order), "Return multiple expert results
+ *           to the same token" (Top-2 weighted sum), "Equal expert counts can
+ *           receive different token counts" (unequal per-expert/per-rank
+ *           counts).
+ *  [NEURON] "Expert Parallelism (EP)" (vLLM on Neuron): "Weight Layout Across
+ *           Ranks" and "Limitations" 1, 3, 4 (E divisible by the EP degree;
+ *           rank r owns experts [r*E/R, (r+1)*E/R), contiguous placement);
+ *           "Router Weights" (every rank scores all E experts).
+ *  [SWIGLU] Shazeer, "GLU Variants Improve Transformer" (2020): the expert
+ *           MLP y = (SiLU(x Wg) * (x Wu)) Wd.
+ *
+ * Conventions for every call:
+ *  - T tokens, H hidden, I intermediate, E experts, k experts per token
+ *    (1 <= k <= min(E, 8)), R logical EP ranks (E % R == 0), S = T*k slots.
+ *    Slot s = t*k + j is token t's j-th choice.
+ *  - All array arguments are DEVICE pointers owned by the caller, row-major;
+ *    activation and weight buffers (and the workspace) 16-byte aligned,
+ *    int32/float32 index and weight arrays 4-byte aligned.  The library never allocates, frees or copies to the
+ *    host, and never synchronises, except moe_get_error.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    enqueued asynchronously on it.
+ *  - Invalid arguments are rejected on the host before anything is enqueued
+ *    (MOE_ERR_INVALID_ARG; moe_last_error_message() names the argument).
+ *    A failed launch returns MOE_ERR_CUDA.
+ *  - Data-dependent problems found on the device (an expert id outside
+ *    [0, E), inconsistent expert offsets, a row index out of range, a
+ *    bounded wait that ran out) never fault: the offending item is skipped,
+ *    a bit is set in a per-device error word, and moe_get_error() reports it.
+ *  - dtype is MOE_F32 (float32) or MOE_BF16 (bfloat16) for activations and
+ *    expert weights; logits and combination weights are always float32;
+ *    all accumulation is float32.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* rejected on the host, nothing enqueued */
+  MOE_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE = 4,      /* the device flagged bad data (see moe_get_error) */
+  MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out */
+} moe_status;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Version of this ABI (bumped on any signature change). */
+int moe_abi_version(void);
+
+/* Static text for a status code. */
+const char* moe_status_string(int status);
+
+/* Text describing the last non-OK status returned on this host thread. */
+const char* moe_last_error_message(void);
+
+/*
+ * moe_route -- [EPRT] "Send tokens ...": each token picks its experts from
+ * all E scores; "Return multiple ...": the combination weights are kept apart
+ * from the choice.  Weight rule: softmax over the k selected logits (k = 1
+ * gives exactly 1.0).
+ *   logits   [T, E] float32 (router affinities, finite)
+ *   topk_ids [T, k] int32   out: experts by logit descending; equal logits
+ *                                (-0 == +0) put the lower id first
+ *   topk_w   [T, k] float32 out: exp(l_j - l_0) / sum_i exp(l_i - l_0)
+ * Constraints: T >= 0, 1 <= E <= 1024, 1 <= k <= min(E, 8).
+ */
+moe_status moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w,
+                     void* stream);
+
+/*
+ * Bytes of device workspace moe_dispatch needs for these sizes.  The
+ * workspace must be zero-filled once before its first use; each call leaves
+ * it ready for the next.  Calls sharing a workspace must not overlap.
+ */
+size_t moe_dispatch_workspace_bytes(int T, int k, int E, int R);
+
+/*
+ * moe_dispatch -- [EPRT] "Send tokens ...": dispatch groups token vectors by
+ * selected expert and tracks each row's source token; [NEURON] "Limitations"
+ * 3-4: rank r owns experts [r*E/R, (r+1)*E/R), so expert-major order is also
+ * rank-major, the layout of an all-to-all send buffer.
+ *   x                 [T, H] dtype     token rows
+ *   topk_ids          [T, k] int32     from moe_route
+ *   x_disp            [S, H] dtype     out: x_disp[slot_to_row[s]] = x[s / k]
+ *   expert_counts     [E]     int32    out: rows per expert
+ *   expert_offsets    [E + 1] int32    out: exclusive prefix sum of counts
+ *   rank_counts       [R]     int32    out: rows per logical rank
+ *   rank_offsets      [R + 1] int32    out: exclusive prefix sum
+ *   slot_to_row       [S]     int32    out: row of slot s (-1 if dropped)
+ *   row_to_slot       [S]     int32    out: inverse (-1 past the last row)
+ *   src_expert_counts [R, E]  int32    out (may be NULL): rows of expert e
+ *                                      whose token comes from source rank r;
+ *                                      token t's source rank is t*R/T
+ *                                      (contiguous, as-equal-as-possible
+ *                                      ranges: the all-to-all send splits)
+ *   workspace / workspace_bytes        scratch from moe_dispatch_workspace_bytes
+ * Rows are ordered by (expert, token): stable in token order within each
+ * expert.  Slots with an id outside [0, E) are dropped (not counted,
+ * slot_to_row = -1) and flagged in the device error word.
+ * Constraints: H * sizeof(dtype) % 16 == 0, E % R == 0, E <= 1024,
+ * 1 <= k <= min(E, 8), S < 2^31.
+ */
+moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
+                        void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                        int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
+                        int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_expert_ffn -- [EPRT] "Send tokens ...": each expert's rows are stacked
+ * and multiplied by that expert's weights, with no mixing across rows;
+ * [SWIGLU]:  h = SiLU(x_disp Wg_e) * (x_disp Wu_e),  y_disp = h Wd_e
+ * for every row in expert e's segment [expert_offsets[e], expert_offsets[e+1]).
+ *   x_disp         [S, H] dtype
+ *   w_gate, w_up   [E, H, I] dtype     (expert e's [H, I] matrix at e*H*I)
+ *   w_down         [E, I, H] dtype
+ *   expert_offsets [E + 1] int32       from moe_dispatch (read on the device)
+ *   h              [S, I] dtype        out: SwiGLU activations (rounded to
+ *                                      dtype), the intermediate of the pair
+ *   y_disp         [S, H] dtype        out: expert outputs
+ * Rows outside [expert_offsets[0], expert_offsets[E]) are not written.
+ * bf16 runs on tcgen05 tensor cores (float32 accumulate in TMEM), float32 on
+ * CUDA cores.  Constraints: H % 8 == 0, I % 8 == 0 (bf16); H % 4, I % 4 (f32).
+ */
+moe_status moe_expert_ffn(const void* x_disp, int dtype, const void* w_gate, const void* w_up,
+                          const void* w_down, const int32_t* expert_offsets, int E, int H, int I, int S, void* h,
+                          void* y_disp, void* stream);
+
+/* First half of moe_expert_ffn: h = SiLU(x_disp Wg_e) * (x_disp Wu_e). */
+moe_status moe_ffn_gate_up(const void* x_disp, int dtype, const void* w_gate, const void* w_up,
+                           const int32_t* expert_offsets, int E, int H, int I, int S, void* h, void* stream);
+
+/* Second half of moe_expert_ffn: y_disp = h Wd_e. */
+moe_status moe_ffn_down(const void* h, int dtype, const void* w_down, const int32_t* expert_offsets, int E, int H,
+                        int I, int S, void* y_disp, void* stream);
+
+/*
+ * moe_combine -- [EPRT] "Send tokens ...": results return to their source
+ * tokens in original order; "Return multiple ...": y(t) = sum_j w_j u_j.
+ *   y_disp      [S, H] dtype
+ *   topk_w      [T, k] float32
+ *   slot_to_row [S] int32              from moe_dispatch
+ *   y           [T, H] dtype           out: float32 sum over j = 0..k-1 in
+ *                                      order, rounded once to dtype
+ * A slot whose row is outside [0, S) contributes nothing and is flagged.
+ */
+moe_status moe_combine(const void* y_disp, int dtype, const float* topk_w, const int32_t* slot_to_row, int T, int k,
+                       int H, void* y, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's error word.
+ * Returns MOE_OK, MOE_ERR_DEVICE (bad ids/offsets/rows were skipped),
+ * MOE_ERR_TIMEOUT (a bounded wait ran out; outputs of that call are
+ * incomplete) or MOE_ERR_CUDA.  `*bits_out` (may be NULL) receives the raw
+ * word: 1 bad expert id, 2 bad expert offsets, 4 bad combine row, 8 timeout.
+ */
+moe_status moe_get_error(void* stream, uint32_t* bits_out);
+
+/*
+ * Self-test of the device-side bounded waits (no counterpart on the pages:
+ * failure detection of this library).  Enqueues one kernel whose single
+ * waiting thread waits on a barrier that nothing completes; after limit_us
+ * microseconds (1 .. 1e6) the wait gives up, sets the timeout bit and the
+ * kernel returns, leaving the context usable.  A following moe_get_error()
+ * returns MOE_ERR_TIMEOUT.
+ */
+moe_status moe_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

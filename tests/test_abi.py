@@ -1,0 +1,98 @@
+"""The C-ABI library builds, loads without a GPU, exports every function that
+include/moe_b200.h declares, and rejects bad arguments on the host before any
+CUDA call (these calls return before touching the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from token_dispatch_combine_b200 import _native
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe_b200.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(moe_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_round_trip_calls():
+    names = declared_functions()
+    for required in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_get_error",
+                     "moe_dispatch_workspace_bytes"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _native.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_native.EXPORTS) <= set(declared_functions())
+
+
+def test_version_and_status_strings():
+    lib = _native.lib()
+    assert lib.moe_abi_version() >= 1
+    assert lib.moe_status_string(0) == b"ok"
+    assert lib.moe_status_string(_native.MOE_ERR_TIMEOUT) == b"device wait timed out"
+
+
+def test_workspace_query_is_host_only():
+    lib = _native.lib()
+    n = lib.moe_dispatch_workspace_bytes(4096, 4, 32, 8)
+    # control word + two [chunks, E] tables + one int per slot
+    assert n >= 256 + 4 * 4096 * 4
+    assert lib.moe_dispatch_workspace_bytes(-1, 4, 32, 8) == 0
+
+
+FAKE = 0x1000  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("T,E,k", [(-1, 4, 1), (4, 0, 1), (4, 4, 0), (4, 4, 5), (4, 2000, 1), (4, 16, 9)])
+def test_route_rejects_bad_sizes(T, E, k):
+    st = _native.lib().moe_route(FAKE, T, E, k, FAKE, FAKE, None)
+    assert st == _native.MOE_ERR_INVALID_ARG
+
+
+def test_route_rejects_misaligned_pointer():
+    lib = _native.lib()
+    assert lib.moe_route(FAKE + 2, 4, 8, 2, FAKE, FAKE, None) == _native.MOE_ERR_INVALID_ARG
+    assert b"logits" in lib.moe_last_error_message()
+
+
+def _dispatch(**kw):
+    a = dict(x=FAKE, dtype=1, T=8, H=64, ids=FAKE, k=2, E=8, R=2, ws_bytes=1 << 20)
+    a.update(kw)
+    return _native.lib().moe_dispatch(a["x"], a["dtype"], a["T"], a["H"], a["ids"], a["k"], a["E"], a["R"], FAKE,
+                                      FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,needle", [
+    (dict(E=9, R=2), b"divide E"),                 # experts must split evenly over ranks
+    (dict(H=60), b"multiple of 16"),               # 120-byte rows break 16-byte vectors
+    (dict(dtype=7), b"dtype"),
+    (dict(k=3, E=2, R=1), b"k must"),
+    (dict(ws_bytes=16), b"workspace_bytes"),
+    (dict(x=FAKE + 8), b"x is not"),
+])
+def test_dispatch_rejects(kw, needle):
+    assert _dispatch(**kw) == _native.MOE_ERR_INVALID_ARG
+    assert needle in _native.lib().moe_last_error_message()
+
+
+def test_ffn_and_combine_reject():
+    lib = _native.lib()
+    # bf16 needs H, I multiples of 8 (16-byte rows for TMA)
+    assert lib.moe_expert_ffn(FAKE, 1, FAKE, FAKE, FAKE, FAKE, 4, 68, 64, 16, FAKE, FAKE, None) == 1
+    assert lib.moe_ffn_gate_up(FAKE, 1, FAKE, FAKE, FAKE, 0, 64, 64, 16, FAKE, None) == 1
+    assert lib.moe_ffn_down(FAKE, 1, FAKE, None, 4, 64, 64, 16, FAKE, None) == 1
+    assert lib.moe_combine(FAKE, 1, FAKE, FAKE, 4, 9, 64, FAKE, None) == 1
+    assert lib.moe_combine(FAKE, 0, FAKE, FAKE, 4, 2, 6, FAKE, None) == 1
+
+
+def test_python_wrapper_raises_moe_error():
+    with pytest.raises(_native.MoeError):
+        _native.check(_native.lib().moe_route(FAKE, 4, 4, 9, FAKE, FAKE, None), "moe_route")

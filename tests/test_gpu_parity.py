@@ -1,0 +1,156 @@
+"""GPU round trip (through the C ABI) against the CPU oracle.
+
+Integer outputs (ids, counts, offsets, permutation, dispatched rows) must be
+bit-exact; combination weights within 1e-6; float outputs within the
+normwise bound max|gpu - oracle| / max|oracle| <= 1e-4 (float32 layers) or
+2e-2 (bf16 layers, float32 accumulation).
+
+Small layers are checked element by element everywhere; the five full-size
+layers are checked in full for routing and dispatch and on sampled rows and
+tokens for the FFN and combine (the oracle computes those one by one)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.gpu_layer import TOL, DeviceLayer, dev_to_np, expert_of_rows, rel_err, widen
+
+pytestmark = pytest.mark.gpu
+
+W = synth.Workload
+SMALL = {
+    "toy_fp32": synth.WORKLOADS["toy_fp32"],
+    # several 128-row tiles per hot expert, zero-row experts (Zipf skew)
+    "bf16_multi_tile": W("bf16_multi_tile", T=512, H=256, I=384, E=8, k=2, R=4, dtype="bf16", seed=11,
+                         bias="zipf1.2"),
+    # K tails (H = 200 = 3*64 + 8), h column tail (I = 200), odd T
+    "bf16_ragged": W("bf16_ragged", T=333, H=200, I=200, E=6, k=3, R=3, dtype="bf16", seed=12, bias="normal0.5"),
+    # down-projection N tail (H = 320 -> 192-wide tiles), I = 136, k = 4 over 16 experts
+    "bf16_ragged_n": W("bf16_ragged_n", T=257, H=320, I=136, E=16, k=4, R=4, dtype="bf16", seed=13),
+    "bf16_one_token": W("bf16_one_token", T=1, H=64, I=64, E=4, k=1, R=2, dtype="bf16", seed=14),
+    "f32_top4": W("f32_top4", T=100, H=96, I=160, E=8, k=4, R=2, dtype="f32", seed=15),
+    "bf16_top8_e256": W("bf16_top8_e256", T=96, H=128, I=128, E=256, k=8, R=32, dtype="bf16", seed=16),
+}
+
+
+def run_gpu(layer: DeviceLayer, rt=None):
+    from token_dispatch_combine_b200 import MoERoundTrip, moe_get_error
+    wl = layer.wl
+    if rt is None:
+        rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, layer.x_dev.dtype)
+    rt.forward(layer.x_dev, layer.logits_dev, layer.w_gate, layer.w_up, layer.w_down)
+    st, bits = moe_get_error()
+    assert st == 0 and bits == 0, (st, bits)
+    return rt
+
+
+def check_routing_and_dispatch(layer: DeviceLayer, rt):
+    wl = layer.wl
+    ids, w = oracle.route(layer.logits, wl.k)
+    assert (dev_to_np(rt.topk_ids) == ids).all()
+    np.testing.assert_allclose(dev_to_np(rt.topk_w), w, rtol=0, atol=1e-6)
+    ref = oracle.dispatch_index(ids, wl.E, wl.R)
+    for name in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "slot_to_row", "row_to_slot",
+                 "src_expert_counts"):
+        got = dev_to_np(getattr(rt.disp, name))
+        assert (got == ref[name]).all(), name
+    x_disp = oracle.dispatch_rows(layer.x, wl.k, ref["slot_to_row"])
+    assert (dev_to_np(rt.disp.x_disp) == x_disp).all()
+    return ids, w, ref, x_disp
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_layer_full_parity(name):
+    wl = SMALL[name]
+    layer = DeviceLayer(wl)
+    rt = run_gpu(layer)
+    ids, w, ref, x_disp = check_routing_and_dispatch(layer, rt)
+    n = int(ref["expert_offsets"][-1])
+    row_expert = expert_of_rows(ref["expert_offsets"], np.arange(n))
+    g, u, d = layer.host_weights(range(wl.E))
+    y_ref, a_ref = oracle.ffn_rows(x_disp[:n], row_expert, g, u, d, wl.H, wl.I, want_act=True)
+    tol = TOL[wl.dtype]
+    assert rel_err(dev_to_np(rt.h)[:n], a_ref) <= tol
+    assert rel_err(dev_to_np(rt.y_disp)[:n], y_ref) <= tol
+    y = oracle.combine(y_ref, w, ref["slot_to_row"])
+    assert rel_err(dev_to_np(rt.y), y) <= tol
+
+
+def _sample_rows(offsets, counts, S, rng, n_random=24):
+    hot = int(np.argmax(counts))
+    rows = {0, S - 1, int(offsets[hot]), int(offsets[hot + 1]) - 1}
+    nz = np.nonzero(counts)[0]
+    for e in rng.choice(nz, size=min(4, len(nz)), replace=False):
+        rows |= {int(offsets[e]), int(offsets[e + 1]) - 1}
+    rows |= set(rng.integers(0, S, n_random).tolist())
+    return np.array(sorted(rows), np.int64)
+
+
+@pytest.mark.parametrize("name", ["gptoss_uniform", "gptoss_zipf", "dsr1_decode", "dsr1_prefill"])
+def test_full_size_layer(name):
+    wl = synth.WORKLOADS[name]
+    layer = DeviceLayer(wl)
+    rt = run_gpu(layer)
+    ids, w, ref, x_disp = check_routing_and_dispatch(layer, rt)
+    rng = np.random.default_rng(wl.seed)
+    S = wl.S
+    rows = _sample_rows(ref["expert_offsets"], ref["expert_counts"], S, rng)
+    tokens = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 6)]))
+    tok_rows = ref["slot_to_row"].reshape(wl.T, wl.k)[tokens].ravel()
+    all_rows = np.unique(np.concatenate([rows, tok_rows]))
+    experts = expert_of_rows(ref["expert_offsets"], all_rows)
+    g, u, d = layer.host_weights(experts)
+    y_rows, a_rows = oracle.ffn_rows(x_disp[all_rows], experts, g, u, d, wl.H, wl.I, want_act=True)
+    tol = TOL[wl.dtype]
+    h_gpu = dev_to_np(rt.h[torch.from_numpy(all_rows).cuda()])
+    yd_gpu = dev_to_np(rt.y_disp[torch.from_numpy(all_rows).cuda()])
+    assert rel_err(h_gpu, a_rows) <= tol
+    assert rel_err(yd_gpu, y_rows) <= tol
+    # combine on the sampled tokens: their k rows, renumbered into the sample
+    pos = {int(r): i for i, r in enumerate(all_rows)}
+    mini_s2r = np.array([pos[int(r)] for r in tok_rows], np.int32)
+    y_ref = oracle.combine(y_rows, w[tokens], mini_s2r)
+    y_gpu = dev_to_np(rt.y[torch.from_numpy(tokens).cuda()])
+    assert rel_err(y_gpu, y_ref) <= tol
+    # every token's output is finite
+    assert torch.isfinite(rt.y.float()).all()
+
+
+def test_repeated_calls_are_identical():
+    wl = SMALL["bf16_multi_tile"]
+    layer = DeviceLayer(wl)
+    rt = run_gpu(layer)
+    first = [dev_to_np(t).copy() for t in (rt.disp.x_disp, rt.h, rt.y_disp, rt.y)]
+    run_gpu(layer, rt)  # workspace reused: the control word must have been reset
+    for a, t in zip(first, (rt.disp.x_disp, rt.h, rt.y_disp, rt.y)):
+        assert (a == dev_to_np(t)).all()
+
+
+def test_all_tokens_to_one_expert():
+    wl = W("one_hot", T=300, H=128, I=128, E=8, k=1, R=2, dtype="bf16", seed=17)
+    logits = np.zeros((wl.T, wl.E), np.float32)
+    logits[:, 5] = 1.0
+    layer = DeviceLayer(wl, logits=logits)
+    rt = run_gpu(layer)
+    _, _, ref, _ = check_routing_and_dispatch(layer, rt)
+    assert ref["expert_counts"].tolist() == [0, 0, 0, 0, 0, 300, 0, 0]
+    x = widen(layer.x)
+    # y = FFN_5(x) for every token; compare with the oracle row by row
+    g, u, d = layer.host_weights([5])
+    y_ref = oracle.ffn_rows(layer.x, np.full(wl.T, 5, np.int32), g, u, d, wl.H, wl.I)
+    assert rel_err(dev_to_np(rt.y), y_ref) <= TOL["bf16"]
+    assert np.isfinite(x).all()
+
+
+def test_identity_experts_combine_reproduces_input():
+    """combine(dispatch(x)) with y_disp := x_disp and weights summing to one gives x back."""
+    from token_dispatch_combine_b200 import MoERoundTrip, moe_combine
+    wl = W("ident", T=200, H=64, I=64, E=8, k=4, R=4, dtype="f32", seed=18)
+    layer = DeviceLayer(wl)
+    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, torch.float32)
+    rt.route(layer.logits_dev)
+    rt.dispatch(layer.x_dev)
+    y = torch.empty_like(layer.x_dev)
+    moe_combine(rt.disp.x_disp, rt.topk_w, rt.disp.slot_to_row, y)
+    np.testing.assert_allclose(dev_to_np(y), layer.x, rtol=0, atol=1e-6 * np.abs(layer.x).max())

@@ -1,0 +1,19 @@
+"""MoE expert-parallel token round trip on one B200 (sm_100a).
+
+route -> dispatch -> grouped SwiGLU expert FFN -> combine, as hand-written
+CUDA kernels behind the C ABI of include/moe_b200.h.  This package is the
+ctypes binding of that library (``_native``) plus torch-facing wrappers with
+the same names (``api``).  Importing it builds/loads the library and raises
+if that is impossible: there is no other implementation to fall back to.
+"""
+from . import _native
+from .api import (DispatchOut, MoERoundTrip, moe_combine, moe_dispatch, moe_dispatch_workspace_bytes, moe_expert_ffn,
+                  moe_ffn_down, moe_ffn_gate_up, moe_get_error, moe_route, new_dispatch_workspace)
+from ._native import MoeError
+
+_native.lib()  # build (if needed) and load now: fail loudly at import
+
+__all__ = [
+    "DispatchOut", "MoERoundTrip", "MoeError", "moe_combine", "moe_dispatch", "moe_dispatch_workspace_bytes",
+    "moe_expert_ffn", "moe_ffn_down", "moe_ffn_gate_up", "moe_get_error", "moe_route", "new_dispatch_workspace",
+]

@@ -1,0 +1,75 @@
+"""ctypes binding of libmoe_b200.so (declared in include/moe_b200.h).
+
+Argument marshalling only: every step of the round trip runs in the CUDA
+library.  There is no fallback -- if the library cannot be built or loaded,
+importing the package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+from . import build as _build
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT = range(6)
+MOE_F32, MOE_BF16 = 0, 1
+
+# error-word bits reported by moe_get_error
+ERR_BAD_ID, ERR_BAD_OFFSETS, ERR_BAD_ROW, ERR_TIMEOUT = 1, 2, 4, 8
+
+EXPORTS = (
+    "moe_abi_version", "moe_status_string", "moe_last_error_message", "moe_route", "moe_dispatch_workspace_bytes",
+    "moe_dispatch", "moe_expert_ffn", "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_get_error", "moe_selftest_wait_timeout",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, fn: str, msg: str):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status}: {msg}")
+
+
+def _configure(lib):
+    vp, i32, sz, u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
+    sigs = {
+        "moe_abi_version": ([], i32),
+        "moe_status_string": ([i32], ctypes.c_char_p),
+        "moe_last_error_message": ([], ctypes.c_char_p),
+        "moe_route": ([vp, i32, i32, i32, vp, vp, vp], i32),
+        "moe_dispatch_workspace_bytes": ([i32, i32, i32, i32], sz),
+        "moe_dispatch": ([vp, i32, i32, i32, vp, i32, i32, i32] + [vp] * 8 + [vp, sz, vp], i32),
+        "moe_expert_ffn": ([vp, i32, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp], i32),
+        "moe_ffn_gate_up": ([vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp], i32),
+        "moe_ffn_down": ([vp, i32, vp, vp, i32, i32, i32, i32, vp, vp], i32),
+        "moe_combine": ([vp, i32, vp, vp, i32, i32, i32, vp, vp], i32),
+        "moe_get_error": ([vp, u32p], i32),
+        "moe_selftest_wait_timeout": ([ctypes.c_uint, vp], i32),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+def lib():
+    """The loaded library (built in-tree first if missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            _lib = _configure(ctypes.CDLL(path))
+    return _lib
+
+
+def check(status: int, fn: str):
+    if status != MOE_OK:
+        msg = lib().moe_last_error_message().decode(errors="replace")
+        raise MoeError(status, fn, msg)
+
+
+def library_path() -> str:
+    return _build.LIB_PATH

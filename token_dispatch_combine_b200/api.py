@@ -1,0 +1,193 @@
+"""Torch-facing wrappers of the C ABI: same names as the C calls, argument
+marshalling only (device pointers, sizes, the current CUDA stream).
+
+PyTorch supplies device memory and streams; every step of the round trip
+runs in libmoe_b200.so.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _native
+from ._native import MOE_BF16, MOE_F32, check
+
+_DT = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None, name: str, dtype=None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"activations/weights must be float32 or bfloat16, got {t.dtype}")
+    return _DT[t.dtype]
+
+
+def moe_route(logits: torch.Tensor, k: int, topk_ids: torch.Tensor | None = None, topk_w: torch.Tensor | None = None,
+              stream=None):
+    """Top-k expert ids [T,k] int32 and softmax-over-top-k weights [T,k] float32."""
+    T, E = logits.shape
+    if topk_ids is None:
+        topk_ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    check(_native.lib().moe_route(_ptr(logits, "logits", torch.float32), T, E, k, _ptr(topk_ids, "topk_ids", torch.int32),
+                                  _ptr(topk_w, "topk_w", torch.float32), _stream(stream)), "moe_route")
+    return topk_ids, topk_w
+
+
+def moe_dispatch_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
+    return int(_native.lib().moe_dispatch_workspace_bytes(T, k, E, R))
+
+
+@dataclass
+class DispatchOut:
+    x_disp: torch.Tensor
+    expert_counts: torch.Tensor
+    expert_offsets: torch.Tensor
+    rank_counts: torch.Tensor
+    rank_offsets: torch.Tensor
+    slot_to_row: torch.Tensor
+    row_to_slot: torch.Tensor
+    src_expert_counts: torch.Tensor | None
+
+    @staticmethod
+    def empty(T, H, k, E, R, dtype, device, src_counts=True) -> "DispatchOut":
+        S = T * k
+        i32 = dict(dtype=torch.int32, device=device)
+        return DispatchOut(
+            x_disp=torch.empty((S, H), dtype=dtype, device=device),
+            expert_counts=torch.empty(E, **i32), expert_offsets=torch.empty(E + 1, **i32),
+            rank_counts=torch.empty(R, **i32), rank_offsets=torch.empty(R + 1, **i32),
+            slot_to_row=torch.empty(S, **i32), row_to_slot=torch.empty(S, **i32),
+            src_expert_counts=torch.empty((R, E), **i32) if src_counts else None)
+
+
+def new_dispatch_workspace(T: int, k: int, E: int, R: int, device) -> torch.Tensor:
+    """Zero-filled workspace of moe_dispatch_workspace_bytes() bytes."""
+    return torch.zeros(moe_dispatch_workspace_bytes(T, k, E, R), dtype=torch.uint8, device=device)
+
+
+def moe_dispatch(x: torch.Tensor, topk_ids: torch.Tensor, E: int, R: int, out: DispatchOut, workspace: torch.Tensor,
+                 stream=None) -> DispatchOut:
+    T, H = x.shape
+    k = topk_ids.shape[1]
+    i32 = torch.int32
+    check(_native.lib().moe_dispatch(
+        _ptr(x, "x"), _dtype(x), T, H, _ptr(topk_ids, "topk_ids", i32), k, E, R, _ptr(out.x_disp, "x_disp", x.dtype),
+        _ptr(out.expert_counts, "expert_counts", i32), _ptr(out.expert_offsets, "expert_offsets", i32),
+        _ptr(out.rank_counts, "rank_counts", i32), _ptr(out.rank_offsets, "rank_offsets", i32),
+        _ptr(out.slot_to_row, "slot_to_row", i32), _ptr(out.row_to_slot, "row_to_slot", i32),
+        _ptr(out.src_expert_counts, "src_expert_counts", i32), _ptr(workspace, "workspace", torch.uint8),
+        workspace.numel(), _stream(stream)), "moe_dispatch")
+    return out
+
+
+def moe_ffn_gate_up(x_disp, w_gate, w_up, expert_offsets, h, stream=None):
+    S, H = x_disp.shape
+    E, _, I = w_gate.shape
+    check(_native.lib().moe_ffn_gate_up(
+        _ptr(x_disp, "x_disp"), _dtype(x_disp), _ptr(w_gate, "w_gate", x_disp.dtype), _ptr(w_up, "w_up", x_disp.dtype),
+        _ptr(expert_offsets, "expert_offsets", torch.int32), E, H, I, S, _ptr(h, "h", x_disp.dtype),
+        _stream(stream)), "moe_ffn_gate_up")
+    return h
+
+
+def moe_ffn_down(h, w_down, expert_offsets, y_disp, stream=None):
+    S, I = h.shape
+    E, _, H = w_down.shape
+    check(_native.lib().moe_ffn_down(
+        _ptr(h, "h"), _dtype(h), _ptr(w_down, "w_down", h.dtype), _ptr(expert_offsets, "expert_offsets", torch.int32),
+        E, H, I, S, _ptr(y_disp, "y_disp", h.dtype), _stream(stream)), "moe_ffn_down")
+    return y_disp
+
+
+def moe_expert_ffn(x_disp, w_gate, w_up, w_down, expert_offsets, h, y_disp, stream=None):
+    S, H = x_disp.shape
+    E, _, I = w_gate.shape
+    dt = x_disp.dtype
+    check(_native.lib().moe_expert_ffn(
+        _ptr(x_disp, "x_disp"), _dtype(x_disp), _ptr(w_gate, "w_gate", dt), _ptr(w_up, "w_up", dt),
+        _ptr(w_down, "w_down", dt), _ptr(expert_offsets, "expert_offsets", torch.int32), E, H, I, S,
+        _ptr(h, "h", dt), _ptr(y_disp, "y_disp", dt), _stream(stream)), "moe_expert_ffn")
+    return y_disp
+
+
+def moe_combine(y_disp, topk_w, slot_to_row, y, stream=None):
+    T, H = y.shape
+    k = topk_w.shape[1]
+    check(_native.lib().moe_combine(
+        _ptr(y_disp, "y_disp", y.dtype), _dtype(y), _ptr(topk_w, "topk_w", torch.float32),
+        _ptr(slot_to_row, "slot_to_row", torch.int32), T, k, H, _ptr(y, "y"), _stream(stream)), "moe_combine")
+    return y
+
+
+def moe_get_error(stream=None) -> tuple[int, int]:
+    """Synchronise the stream; return (status, error-word bits) and clear the word."""
+    bits = ctypes.c_uint32(0)
+    st = _native.lib().moe_get_error(_stream(stream), ctypes.byref(bits))
+    return st, bits.value
+
+
+class MoERoundTrip:
+    """Buffers and the four calls of one MoE layer round trip on one GPU.
+
+    Route -> dispatch -> grouped SwiGLU FFN -> combine, all on `stream`.
+    Device memory for every intermediate is allocated once here (through
+    torch); ``forward`` enqueues six kernels and allocates nothing.
+    """
+
+    def __init__(self, T, H, I, E, k, R, dtype, device="cuda", src_counts=True):
+        self.T, self.H, self.I, self.E, self.k, self.R = T, H, I, E, k, R
+        self.dtype = dtype
+        self.device = torch.device(device)
+        S = T * k
+        self.topk_ids = torch.empty((T, k), dtype=torch.int32, device=self.device)
+        self.topk_w = torch.empty((T, k), dtype=torch.float32, device=self.device)
+        self.disp = DispatchOut.empty(T, H, k, E, R, dtype, self.device, src_counts)
+        self.workspace = new_dispatch_workspace(T, k, E, R, self.device)
+        self.h = torch.empty((S, I), dtype=dtype, device=self.device)
+        self.y_disp = torch.empty((S, H), dtype=dtype, device=self.device)
+        self.y = torch.empty((T, H), dtype=dtype, device=self.device)
+
+    def route(self, logits, stream=None):
+        return moe_route(logits, self.k, self.topk_ids, self.topk_w, stream)
+
+    def dispatch(self, x, stream=None):
+        return moe_dispatch(x, self.topk_ids, self.E, self.R, self.disp, self.workspace, stream)
+
+    def gate_up(self, w_gate, w_up, stream=None):
+        return moe_ffn_gate_up(self.disp.x_disp, w_gate, w_up, self.disp.expert_offsets, self.h, stream)
+
+    def down(self, w_down, stream=None):
+        return moe_ffn_down(self.h, w_down, self.disp.expert_offsets, self.y_disp, stream)
+
+    def combine(self, stream=None):
+        return moe_combine(self.y_disp, self.topk_w, self.disp.slot_to_row, self.y, stream)
+
+    def forward(self, x, logits, w_gate, w_up, w_down, stream=None):
+        self.route(logits, stream)
+        self.dispatch(x, stream)
+        self.gate_up(w_gate, w_up, stream)
+        self.down(w_down, stream)
+        return self.combine(stream)
+
+    KERNELS_PER_FORWARD = 6  # route, dispatch x2, gate/up, down, combine

@@ -1,0 +1,233 @@
+// C ABI of the MoE round trip (declared in include/moe_b200.h).
+//
+// Host side only validates arguments, picks kernel configurations and
+// enqueues launches on the caller's stream.  It never allocates, never copies
+// to the host and never synchronises (moe_get_error excepted).
+#include <cstdio>
+#include <string>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "ffn_simt.cuh"
+#include "ffn_tc.cuh"
+#include "route.cuh"
+
+namespace {
+
+thread_local std::string g_last_msg;
+
+moe_status fail(moe_status st, const std::string& msg) {
+  g_last_msg = msg;
+  return st;
+}
+
+moe_status cuda_status(cudaError_t err, const char* where) {
+  if (err == cudaSuccess) return MOE_OK;
+  return fail(MOE_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(err));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t dtype_size(int dt) { return dt == MOE_F32 ? 4 : dt == MOE_BF16 ? 2 : 0; }
+
+#define MOE_REQUIRE(cond, msg)                                   \
+  do {                                                           \
+    if (!(cond)) return fail(MOE_ERR_INVALID_ARG, (msg));        \
+  } while (0)
+
+#define MOE_REQUIRE_PTR(p, a, name)                                                              \
+  do {                                                                                           \
+    MOE_REQUIRE((p) != nullptr, std::string(name) + " is NULL");                                 \
+    MOE_REQUIRE(aligned((p), (a)), std::string(name) + " is not " #a "-byte aligned");           \
+  } while (0)
+
+moe_status check_k_e(int k, int E) {
+  MOE_REQUIRE(E >= 1 && E <= 1024, "E must be in [1, 1024]");
+  MOE_REQUIRE(k >= 1 && k <= 8 && k <= E, "k must be in [1, min(E, 8)]");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK:
+      return "ok";
+    case MOE_ERR_INVALID_ARG:
+      return "invalid argument";
+    case MOE_ERR_UNSUPPORTED:
+      return "unsupported";
+    case MOE_ERR_CUDA:
+      return "CUDA error";
+    case MOE_ERR_DEVICE:
+      return "device flagged bad data";
+    case MOE_ERR_TIMEOUT:
+      return "device wait timed out";
+    default:
+      return "unknown status";
+  }
+}
+
+const char* moe_last_error_message(void) { return g_last_msg.c_str(); }
+
+moe_status moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids, float* topk_w, void* stream) {
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  moe_status st = check_k_e(k, E);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(logits, 4, "logits");
+  MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
+  MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
+  return cuda_status(moe::launch_route(logits, T, E, k, topk_ids, topk_w, (cudaStream_t)stream), "moe_route");
+}
+
+size_t moe_dispatch_workspace_bytes(int T, int k, int E, int R) {
+  if (T < 0 || k < 1 || E < 1 || R < 1) return 0;
+  return moe::dispatch_ws_bytes(moe::make_dispatch_geom(T, k, E, R));
+}
+
+moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
+                        void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                        int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
+                        int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream) {
+  const size_t es = dtype_size(dtype);
+  MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  MOE_REQUIRE(H >= 1 && (H * es) % 16 == 0, "H * sizeof(dtype) must be a positive multiple of 16");
+  moe_status st = check_k_e(k, E);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(R >= 1 && E % R == 0, "R must be >= 1 and divide E");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  MOE_REQUIRE_PTR(expert_counts, 4, "expert_counts");
+  MOE_REQUIRE_PTR(expert_offsets, 4, "expert_offsets");
+  MOE_REQUIRE_PTR(rank_counts, 4, "rank_counts");
+  MOE_REQUIRE_PTR(rank_offsets, 4, "rank_offsets");
+  MOE_REQUIRE(src_expert_counts == nullptr || aligned(src_expert_counts, 4), "src_expert_counts misaligned");
+  MOE_REQUIRE_PTR(workspace, 16, "workspace");
+  const moe::DispatchGeom g = moe::make_dispatch_geom(T, k, E, R);
+  MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(g), "workspace_bytes smaller than moe_dispatch_workspace_bytes()");
+  if (T > 0) {
+    MOE_REQUIRE_PTR(x, 16, "x");
+    MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
+    MOE_REQUIRE_PTR(x_disp, 16, "x_disp");
+    MOE_REQUIRE_PTR(slot_to_row, 4, "slot_to_row");
+    MOE_REQUIRE_PTR(row_to_slot, 4, "row_to_slot");
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = moe::launch_dispatch(g, H, (const __nv_bfloat16*)x, topk_ids, workspace, (__nv_bfloat16*)x_disp,
+                               expert_counts, expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
+                               src_expert_counts, s);
+  else
+    err = moe::launch_dispatch(g, H, (const float*)x, topk_ids, workspace, (float*)x_disp, expert_counts,
+                               expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
+                               src_expert_counts, s);
+  return cuda_status(err, "moe_dispatch");
+}
+
+static moe_status check_ffn(int dtype, int E, int H, int I, int S, const void* a, const char* a_name,
+                            const int32_t* off) {
+  const size_t es = dtype_size(dtype);
+  MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(E >= 1 && E <= 1024, "E must be in [1, 1024]");
+  MOE_REQUIRE(H >= 1 && I >= 1, "H and I must be >= 1");
+  MOE_REQUIRE((H * es) % 16 == 0 && (I * es) % 16 == 0, "H * sizeof(dtype) and I * sizeof(dtype) must be multiples of 16");
+  MOE_REQUIRE(S >= 0, "S must be >= 0");
+  MOE_REQUIRE_PTR(off, 4, "expert_offsets");
+  if (S > 0) MOE_REQUIRE_PTR(a, 16, a_name);
+  return MOE_OK;
+}
+
+moe_status moe_ffn_gate_up(const void* x_disp, int dtype, const void* w_gate, const void* w_up,
+                           const int32_t* expert_offsets, int E, int H, int I, int S, void* h, void* stream) {
+  moe_status st = check_ffn(dtype, E, H, I, S, x_disp, "x_disp", expert_offsets);
+  if (st != MOE_OK) return st;
+  if (S == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(w_gate, 16, "w_gate");
+  MOE_REQUIRE_PTR(w_up, 16, "w_up");
+  MOE_REQUIRE_PTR(h, 16, "h");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = moe::tc::launch_gate_up(x_disp, w_gate, w_up, expert_offsets, E, H, I, S, h, s);
+  else
+    err = moe::launch_ffn_simt_gate_up((const float*)x_disp, (const float*)w_gate, (const float*)w_up,
+                                       expert_offsets, E, H, I, S, (float*)h, s);
+  return cuda_status(err, "moe_ffn_gate_up");
+}
+
+moe_status moe_ffn_down(const void* h, int dtype, const void* w_down, const int32_t* expert_offsets, int E, int H,
+                        int I, int S, void* y_disp, void* stream) {
+  moe_status st = check_ffn(dtype, E, H, I, S, h, "h", expert_offsets);
+  if (st != MOE_OK) return st;
+  if (S == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(w_down, 16, "w_down");
+  MOE_REQUIRE_PTR(y_disp, 16, "y_disp");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = moe::tc::launch_down(h, w_down, expert_offsets, E, H, I, S, y_disp, s);
+  else
+    err = moe::launch_ffn_simt_down((const float*)h, (const float*)w_down, expert_offsets, E, H, I, S,
+                                    (float*)y_disp, s);
+  return cuda_status(err, "moe_ffn_down");
+}
+
+moe_status moe_expert_ffn(const void* x_disp, int dtype, const void* w_gate, const void* w_up,
+                          const void* w_down, const int32_t* expert_offsets, int E, int H, int I, int S, void* h,
+                          void* y_disp, void* stream) {
+  moe_status st = moe_ffn_gate_up(x_disp, dtype, w_gate, w_up, expert_offsets, E, H, I, S, h, stream);
+  if (st != MOE_OK) return st;
+  return moe_ffn_down(h, dtype, w_down, expert_offsets, E, H, I, S, y_disp, stream);
+}
+
+moe_status moe_combine(const void* y_disp, int dtype, const float* topk_w, const int32_t* slot_to_row, int T, int k,
+                       int H, void* y, void* stream) {
+  const size_t es = dtype_size(dtype);
+  MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  MOE_REQUIRE(k >= 1 && k <= 8, "k must be in [1, 8]");
+  MOE_REQUIRE(H >= 1 && (H * es) % 16 == 0, "H * sizeof(dtype) must be a positive multiple of 16");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(y_disp, 16, "y_disp");
+  MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
+  MOE_REQUIRE_PTR(slot_to_row, 4, "slot_to_row");
+  MOE_REQUIRE_PTR(y, 16, "y");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = moe::launch_combine((const __nv_bfloat16*)y_disp, topk_w, slot_to_row, T, k, H, (__nv_bfloat16*)y, s);
+  else
+    err = moe::launch_combine((const float*)y_disp, topk_w, slot_to_row, T, k, H, (float*)y, s);
+  return cuda_status(err, "moe_combine");
+}
+
+moe_status moe_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  MOE_REQUIRE(limit_us >= 1 && limit_us <= 1000000u, "limit_us must be in [1, 1000000]");
+  moe::tc::wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull);
+  return cuda_status(cudaGetLastError(), "moe_selftest_wait_timeout");
+}
+
+moe_status moe_get_error(void* stream, uint32_t* bits_out) {
+  cudaError_t err = cudaStreamSynchronize((cudaStream_t)stream);
+  if (err != cudaSuccess) return cuda_status(err, "moe_get_error: stream synchronize");
+  uint32_t word = 0;
+  err = cudaMemcpyFromSymbol(&word, moe::g_error_word, sizeof(word));
+  if (err != cudaSuccess) return cuda_status(err, "moe_get_error: read error word");
+  if (bits_out) *bits_out = word;
+  if (word == 0) return MOE_OK;
+  const uint32_t zero = 0;
+  err = cudaMemcpyToSymbol(moe::g_error_word, &zero, sizeof(zero));
+  if (err != cudaSuccess) return cuda_status(err, "moe_get_error: clear error word");
+  if (word & moe::kErrTimeout) return fail(MOE_ERR_TIMEOUT, "a bounded device-side wait ran out");
+  return fail(MOE_ERR_DEVICE, "device skipped bad data (error word " + std::to_string(word) + ")");
+}
+
+}  // extern "C"
