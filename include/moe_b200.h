@@ -132,6 +132,33 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
                         int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * moe_dispatch_noalloc -- moe_dispatch for callers that cannot allocate.
+ * (The pages have no counterpart: this is a deployment variant of this
+ * library's dispatch.)
+ *
+ * Same arguments and results as moe_dispatch, without the workspace: some
+ * callers have no way to pass one in and may not call cudaMalloc where they
+ * call us (a host framework that owns all device memory, or a hot path that
+ * must not take cudaMalloc's implicit synchronisation).  The scratch lives in
+ * a fixed array of MOE_DISPATCH_NOALLOC_SCRATCH_BYTES bytes inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  This call allocates nothing and frees nothing.
+ *  - Sizes whose moe_dispatch_workspace_bytes(T, k, E, R) exceeds the
+ *    maximum are rejected with MOE_ERR_INVALID_ARG (use moe_dispatch then).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call on a device shares the one array and finds it as the last
+ *    call left it; the call clears the part that must start at zero.  Calls
+ *    that overlap on the GPU (other streams, other host threads) race on it:
+ *    serialise them.
+ */
+#define MOE_DISPATCH_NOALLOC_SCRATCH_BYTES (2u << 20)
+moe_status moe_dispatch_noalloc(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E,
+                                int R, void* x_disp, int32_t* expert_counts, int32_t* expert_offsets,
+                                int32_t* rank_counts, int32_t* rank_offsets, int32_t* slot_to_row,
+                                int32_t* row_to_slot, int32_t* src_expert_counts, void* stream);
+
+/*
  * moe_expert_ffn -- [EPRT] "Send tokens ...": each expert's rows are stacked
  * and multiplied by that expert's weights, with no mixing across rows;
  * [SWIGLU]:  h = SiLU(x_disp Wg_e) * (x_disp Wu_e),  y_disp = h Wd_e

@@ -47,6 +47,7 @@ def _configure(lib):
         "moe_combine": ([vp, i32, vp, vp, i32, i32, i32, vp, vp], i32),
         "moe_get_error": ([vp, u32p], i32),
         "moe_selftest_wait_timeout": ([ctypes.c_uint, vp], i32),
+        "moe_dispatch_noalloc": ([vp, i32, i32, i32, vp, i32, i32, i32] + [vp] * 8 + [vp], i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)

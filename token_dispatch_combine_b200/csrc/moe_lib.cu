@@ -4,6 +4,7 @@
 // enqueues launches on the caller's stream.  It never allocates, never copies
 // to the host and never synchronises (moe_get_error excepted).
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "combine.cuh"
@@ -129,6 +130,66 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
                                expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
                                src_expert_counts, s);
   return cuda_status(err, "moe_dispatch");
+}
+
+// ---------------------------------------------------------------------------
+// moe_dispatch_noalloc: moe_dispatch with its scratch in a fixed device array.
+//
+// Some callers cannot hand this library a workspace: their own interface has
+// no slot for one, and they may not call cudaMalloc on their execution path
+// (a host framework that owns every allocation, or code that must not risk
+// the implicit device synchronisation and heap growth of cudaMalloc).  For
+// them the dispatch scratch lives in the array below, which the CUDA module
+// reserves on every GPU that loads this library and keeps until the process
+// exits.  Host code never touches the array by name (that name is only a
+// host-side stand-in); its device address is looked up once per device with
+// cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) unsigned char g_dispatch_noalloc_scratch[MOE_DISPATCH_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on the first call there).
+moe_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kNoallocMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "moe_dispatch_noalloc: device index too large");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_dispatch_noalloc_scratch);
+    if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: cudaGetSymbolAddress");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" moe_status moe_dispatch_noalloc(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k,
+                                           int E, int R, void* x_disp, int32_t* expert_counts,
+                                           int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets,
+                                           int32_t* slot_to_row, int32_t* row_to_slot, int32_t* src_expert_counts,
+                                           void* stream) {
+  MOE_REQUIRE(T >= 0 && k >= 1 && E >= 1 && R >= 1, "T >= 0, k >= 1, E >= 1 and R >= 1 are required");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  const size_t need = moe_dispatch_workspace_bytes(T, k, E, R);
+  MOE_REQUIRE(need <= (size_t)MOE_DISPATCH_NOALLOC_SCRATCH_BYTES,
+              "moe_dispatch_noalloc: these sizes need " + std::to_string(need) +
+                  " bytes of scratch, more than the built-in " +
+                  std::to_string((size_t)MOE_DISPATCH_NOALLOC_SCRATCH_BYTES) + "; use moe_dispatch with a workspace");
+  void* scratch = nullptr;
+  moe_status st = noalloc_scratch(&scratch);
+  if (st != MOE_OK) return st;
+  // The array keeps whatever the previous call left; the control word must start at zero.
+  cudaError_t err = cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream);
+  if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: clear control word");
+  return moe_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets, rank_counts,
+                      rank_offsets, slot_to_row, row_to_slot, src_expert_counts, scratch,
+                      (size_t)MOE_DISPATCH_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 static moe_status check_ffn(int dtype, int E, int H, int I, int S, const void* a, const char* a_name,
