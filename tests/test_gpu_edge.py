@@ -154,3 +154,26 @@ def test_bounded_wait_times_out_and_context_survives():
     ids, w = m.moe_route(torch.randn(16, 8, device="cuda"), 2)
     torch.cuda.synchronize()
     assert (dev_to_np(w).sum(1) > 0.999).all()
+
+
+@pytest.mark.parametrize("T,E,k,R", [(2048, 1024, 8, 32),   # count table too big to stage in shared memory
+                                     (100, 64, 8, 8),        # T not a multiple of R
+                                     (5000, 16, 1, 16)])
+def test_dispatch_index_against_oracle(T, E, k, R):
+    m = _api()
+    rng = np.random.default_rng(T + E)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    logits[:, 1] += 1.5  # a hot expert
+    ids, _ = oracle.route(logits, k)
+    x = torch.randn(T, 64, device="cuda", dtype=torch.bfloat16)
+    out = m.DispatchOut.empty(T, 64, k, E, R, torch.bfloat16, "cuda")
+    ws = m.new_dispatch_workspace(T, k, E, R, "cuda")
+    for _ in range(2):  # the workspace must be reusable
+        m.moe_dispatch(x, torch.from_numpy(ids).cuda(), E, R, out, ws)
+        assert m.moe_get_error() == (0, 0)
+        ref = oracle.dispatch_index(ids, E, R)
+        for key in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "slot_to_row", "row_to_slot",
+                    "src_expert_counts"):
+            assert (dev_to_np(getattr(out, key)) == ref[key]).all(), key
+        xd = oracle.dispatch_rows(dev_to_np(x), k, ref["slot_to_row"])
+        assert (dev_to_np(out.x_disp) == xd).all()

@@ -32,7 +32,10 @@ struct DispatchGeom {
   int chunk;    // slots per chunk (= CTA size of kernel 1, a multiple of 32)
   int cpr;      // chunks per source rank
   int nchunks;  // R * cpr
+  int counts_in_smem;  // the last CTA stages the [nchunks][E] counts in shared memory
 };
+
+constexpr size_t kDispatchCountsSmemMax = 96 * 1024;  // bytes of [nchunks][E] counts staged by the last CTA
 
 // First token of source rank r: ceil(r*T/R), so that t*R/T == r on [lo(r), lo(r+1)).
 __host__ __device__ __forceinline__ int src_rank_first_token(int r, int T, int R) {
@@ -55,6 +58,7 @@ inline DispatchGeom make_dispatch_geom(int T, int k, int E, int R) {
   g.cpr = (max_slots + ch - 1) / ch;
   if (g.cpr < 1) g.cpr = 1;
   g.nchunks = R * g.cpr;
+  g.counts_in_smem = (size_t)g.nchunks * E * sizeof(int32_t) <= kDispatchCountsSmemMax;
   return g;
 }
 
@@ -105,8 +109,10 @@ __global__ void __launch_bounds__(1024) dispatch_rank_kernel(
   extern __shared__ int32_t smem_i32[];
   const int nwarps = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = (int)lane_id();
-  int32_t* warp_counts = smem_i32;                     // [nwarps][E]
-  int32_t* scan = smem_i32 + (size_t)nwarps * g.E;      // [E + 1]
+  int32_t* warp_counts = smem_i32;  // [nwarps][E]
+  size_t table = (size_t)nwarps * g.E;
+  if (g.counts_in_smem && (size_t)g.nchunks * g.E > table) table = (size_t)g.nchunks * g.E;
+  int32_t* scan = smem_i32 + table;  // [E + 1]
   __shared__ int s_is_last;
 
   const int c = blockIdx.x;
@@ -150,31 +156,66 @@ __global__ void __launch_bounds__(1024) dispatch_rank_kernel(
   if (!s_is_last) return;
   __threadfence();
 
-  // per expert: running sum over chunks -> chunk bases (relative) and totals
+  // The per-chunk counts come back through L2; every read below is issued
+  // independently of the running sums so that many are in flight at once.
+  const int nce = g.nchunks * g.E;
+  int32_t* cnt = smem_i32;  // warp_counts is dead here: reuse it for the [nchunks][E] counts
+  if (g.counts_in_smem) {
+#pragma unroll 4
+    for (int i = threadIdx.x; i < nce; i += blockDim.x) cnt[i] = __ldcg(ws.chunk_counts + i);
+    __syncthreads();
+  }
+  auto count_at = [&](int cc, int x) {
+    return g.counts_in_smem ? cnt[cc * g.E + x] : __ldcg(ws.chunk_counts + (size_t)cc * g.E + x);
+  };
+  // 1. per-expert totals
   for (int x = threadIdx.x; x < g.E; x += blockDim.x) {
     int run = 0;
-    for (int cc = 0; cc < g.nchunks; ++cc) {
-      const int v = __ldcg(ws.chunk_counts + (size_t)cc * g.E + x);
-      ws.chunk_base[(size_t)cc * g.E + x] = run;
-      run += v;
+    for (int c0 = 0; c0 < g.nchunks; c0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = (c0 + u < g.nchunks) ? count_at(c0 + u, x) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) run += v[u];
     }
     scan[x] = run;
     expert_counts[x] = run;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {  // E <= 1024: a short serial scan
-    int run = 0;
-    for (int x = 0; x < g.E; ++x) {
-      const int v = scan[x];
-      scan[x] = run;
-      run += v;
+  // 2. exclusive scan over experts (warp 0, 32 at a time)
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < g.E; base += 32) {
+      const int v = (base + lane < g.E) ? scan[base + lane] : 0;
+      int incl = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += y;
+      }
+      if (base + lane < g.E) scan[base + lane] = carry + incl - v;
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
-    scan[g.E] = run;
+    if (lane == 0) scan[g.E] = carry;
   }
   __syncthreads();
+  // 3. chunk bases = expert offset + counts of the same expert in earlier chunks
+  for (int x = threadIdx.x; x < g.E; x += blockDim.x) {
+    int run = scan[x];
+    for (int c0 = 0; c0 < g.nchunks; c0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = (c0 + u < g.nchunks) ? count_at(c0 + u, x) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (c0 + u < g.nchunks) {
+          ws.chunk_base[(size_t)(c0 + u) * g.E + x] = run;
+          run += v[u];
+        }
+      }
+    }
+  }
   for (int x = threadIdx.x; x <= g.E; x += blockDim.x) expert_offsets[x] = scan[x];
-  for (size_t i = threadIdx.x; i < (size_t)g.nchunks * g.E; i += blockDim.x)
-    ws.chunk_base[i] += scan[i % g.E];
   const int EL = g.E / g.R;
   for (int r = threadIdx.x; r < g.R; r += blockDim.x) {
     rank_counts[r] = scan[(r + 1) * EL] - scan[r * EL];
@@ -185,7 +226,7 @@ __global__ void __launch_bounds__(1024) dispatch_rank_kernel(
     for (int i = threadIdx.x; i < g.R * g.E; i += blockDim.x) {
       const int r = i / g.E, x = i - r * g.E;
       int sum = 0;
-      for (int ci = 0; ci < g.cpr; ++ci) sum += __ldcg(ws.chunk_counts + (size_t)(r * g.cpr + ci) * g.E + x);
+      for (int ci = 0; ci < g.cpr; ++ci) sum += count_at(r * g.cpr + ci, x);
       src_expert_counts[i] = sum;
     }
   }
@@ -253,7 +294,9 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
                             int32_t* src_expert_counts, cudaStream_t stream) {
   DispatchWs ws = dispatch_ws_carve(workspace, g);
   const int threads1 = g.chunk;
-  const size_t smem1 = sizeof(int32_t) * ((size_t)(threads1 / 32) * g.E + g.E + 1);
+  size_t table = (size_t)(threads1 / 32) * g.E;  // warp_counts, later the staged chunk counts
+  if (g.counts_in_smem && (size_t)g.nchunks * g.E > table) table = (size_t)g.nchunks * g.E;
+  const size_t smem1 = sizeof(int32_t) * (table + g.E + 1);
   if (smem1 > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(dispatch_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem1);

@@ -40,6 +40,21 @@
 
 #include "common.cuh"
 
+// Tuning knobs (compile-time).
+//  MOE_TC_GROUP_M: tiles are visited in groups of this many consecutive m-tiles,
+//    all n-tiles of a group before the next group (0 = plain m-major order).
+//  MOE_TC_HINT_A / MOE_TC_HINT_B: L2 eviction priority of the TMA loads of the
+//    activation and weight tiles (0 normal, 1 evict-first, 2 evict-last).
+#ifndef MOE_TC_GROUP_M
+#define MOE_TC_GROUP_M 0
+#endif
+#ifndef MOE_TC_HINT_A
+#define MOE_TC_HINT_A 0
+#endif
+#ifndef MOE_TC_HINT_B
+#define MOE_TC_HINT_B 0
+#endif
+
 namespace moe {
 namespace tc {
 
@@ -109,6 +124,40 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "[%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+// L2 eviction-priority policy for cache-hinted TMA loads (1 evict-first, 2 evict-last).
+template <int HINT>
+__device__ __forceinline__ uint64_t l2_policy() {
+  uint64_t pol = 0;
+  if (HINT == 1) asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  if (HINT == 2) asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+template <int HINT>
+__device__ __forceinline__ void tma_load_2d_h(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                              uint64_t pol) {
+  if (HINT == 0) {
+    tma_load_2d(dst, map, bar, c0, c1);
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(pol)
+        : "memory");
+  }
+}
+template <int HINT>
+__device__ __forceinline__ void tma_load_3d_h(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                              int c2, uint64_t pol) {
+  if (HINT == 0) {
+    tma_load_3d(dst, map, bar, c0, c1, c2);
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
+        : "memory");
+  }
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -277,7 +326,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // tile -> (expert, first row, end row, first output column)
   auto tile_coords = [&](int tile, int& e, int& m0, int& mend, int& n0) {
-    const int mt = tile / p.ntn, nt = tile - mt * p.ntn;
+    int mt, nt;
+    if (MOE_TC_GROUP_M > 0) {
+      // groups of MOE_TC_GROUP_M m-tiles; inside a group, n-tile-major
+      const int per_group = MOE_TC_GROUP_M * p.ntn;
+      const int g = tile / per_group, r = tile - g * per_group;
+      const int gm = min(MOE_TC_GROUP_M, total_mtiles - g * MOE_TC_GROUP_M);
+      nt = r / gm;
+      mt = g * MOE_TC_GROUP_M + (r - nt * gm);
+    } else {
+      mt = tile / p.ntn;
+      nt = tile - mt * p.ntn;
+    }
     int lo = 0, hi = p.E - 1;  // largest e with s_pre[e] <= mt
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -296,6 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed_mask = 0, armed_par = 0;
       bool ok = true;
+      const uint64_t pol_a = l2_policy<MOE_TC_HINT_A>();
+      const uint64_t pol_b = l2_policy<MOE_TC_HINT_B>();
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         int e, m0, mend, n0;
         tile_coords(tile, e, m0, mend, n0);
@@ -310,17 +372,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           const uint32_t a_dst = smem_u32(sA + (size_t)stage * kABytes);
           const uint32_t b_dst = smem_u32(sB + (size_t)stage * C::kBBytes);
-          tma_load_2d(a_dst, &tmap_a, fb, kb * BK, m0);
+          tma_load_2d_h<MOE_TC_HINT_A>(a_dst, &tmap_a, fb, kb * BK, m0, pol_a);
           if (GATEUP) {
             constexpr int HB = C::NBOX / 2;  // boxes per half
 #pragma unroll
             for (int i = 0; i < HB; ++i) {
-              tma_load_3d(b_dst + i * kBoxBytes, &tmap_b0, fb, n0 + 64 * i, kb * BK, e);
-              tma_load_3d(b_dst + (HB + i) * kBoxBytes, &tmap_b1, fb, n0 + 64 * i, kb * BK, e);
+              tma_load_3d_h<MOE_TC_HINT_B>(b_dst + i * kBoxBytes, &tmap_b0, fb, n0 + 64 * i, kb * BK, e, pol_b);
+              tma_load_3d_h<MOE_TC_HINT_B>(b_dst + (HB + i) * kBoxBytes, &tmap_b1, fb, n0 + 64 * i, kb * BK, e,
+                                           pol_b);
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < C::NBOX; ++i) tma_load_3d(b_dst + i * kBoxBytes, &tmap_b0, fb, n0 + 64 * i, kb * BK, e);
+            for (int i = 0; i < C::NBOX; ++i)
+              tma_load_3d_h<MOE_TC_HINT_B>(b_dst + i * kBoxBytes, &tmap_b0, fb, n0 + 64 * i, kb * BK, e, pol_b);
           }
           if (++stage == STAGES) {
             stage = 0;
