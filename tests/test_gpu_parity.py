@@ -154,3 +154,25 @@ def test_identity_experts_combine_reproduces_input():
     y = torch.empty_like(layer.x_dev)
     moe_combine(rt.disp.x_disp, rt.topk_w, rt.disp.slot_to_row, y)
     np.testing.assert_allclose(dev_to_np(y), layer.x, rtol=0, atol=1e-6 * np.abs(layer.x).max())
+
+
+def test_host_pipeline_matches_forward():
+    """MoEHostPipeline (overlapped upload/compute/download) gives, per batch, exactly
+    what a plain forward of that batch gives."""
+    from token_dispatch_combine_b200 import MoEHostPipeline, MoERoundTrip
+    wl = W("pipe", T=300, H=256, I=384, E=8, k=2, R=4, dtype="bf16", seed=19)
+    layer = DeviceLayer(wl)
+    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, torch.bfloat16)
+    batches, want = [], []
+    for b in range(5):
+        x = torch.randn(wl.T, wl.H, device="cuda").to(torch.bfloat16)
+        lg = torch.randn(wl.T, wl.E, device="cuda")
+        want.append(rt.forward(x, lg, layer.w_gate, layer.w_up, layer.w_down).clone())
+        batches.append((x.view(torch.int16).cpu().pin_memory(), lg.cpu().pin_memory(),
+                        torch.empty(wl.T, wl.H, dtype=torch.int16).pin_memory()))
+    torch.cuda.synchronize()
+    pipe = MoEHostPipeline(rt, layer.w_gate, layer.w_up, layer.w_down)
+    pipe.run(batches).synchronize()
+    torch.cuda.synchronize()
+    for (_, _, yh), y in zip(batches, want):
+        assert torch.equal(yh, y.view(torch.int16).cpu())

@@ -7,13 +7,13 @@ the same names (``api``).  Importing it builds/loads the library and raises
 if that is impossible: there is no other implementation to fall back to.
 """
 from . import _native
-from .api import (DispatchOut, MoERoundTrip, moe_combine, moe_dispatch, moe_dispatch_workspace_bytes, moe_expert_ffn,
+from .api import (DispatchOut, MoEHostPipeline, MoERoundTrip, moe_combine, moe_dispatch, moe_dispatch_workspace_bytes, moe_expert_ffn,
                   moe_ffn_down, moe_ffn_gate_up, moe_get_error, moe_route, new_dispatch_workspace)
 from ._native import MoeError
 
 _native.lib()  # build (if needed) and load now: fail loudly at import
 
 __all__ = [
-    "DispatchOut", "MoERoundTrip", "MoeError", "moe_combine", "moe_dispatch", "moe_dispatch_workspace_bytes",
+    "DispatchOut", "MoEHostPipeline", "MoERoundTrip", "MoeError", "moe_combine", "moe_dispatch", "moe_dispatch_workspace_bytes",
     "moe_expert_ffn", "moe_ffn_down", "moe_ffn_gate_up", "moe_get_error", "moe_route", "new_dispatch_workspace",
 ]

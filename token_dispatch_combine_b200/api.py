@@ -180,14 +180,69 @@ class MoERoundTrip:
     def down(self, w_down, stream=None):
         return moe_ffn_down(self.h, w_down, self.disp.expert_offsets, self.y_disp, stream)
 
-    def combine(self, stream=None):
-        return moe_combine(self.y_disp, self.topk_w, self.disp.slot_to_row, self.y, stream)
+    def combine(self, stream=None, y=None):
+        return moe_combine(self.y_disp, self.topk_w, self.disp.slot_to_row, self.y if y is None else y, stream)
 
-    def forward(self, x, logits, w_gate, w_up, w_down, stream=None):
+    def forward(self, x, logits, w_gate, w_up, w_down, stream=None, y=None):
         self.route(logits, stream)
         self.dispatch(x, stream)
         self.gate_up(w_gate, w_up, stream)
         self.down(w_down, stream)
-        return self.combine(stream)
+        return self.combine(stream, y)
 
     KERNELS_PER_FORWARD = 6  # route, dispatch x2, gate/up, down, combine
+
+
+class MoEHostPipeline:
+    """Round trips over a sequence of host-resident batches.
+
+    Each batch's inputs (x, logits) start in pinned host memory and its output
+    y ends there.  Three CUDA streams overlap the host->device copy of batch
+    i+1 and the device->host copy of batch i-1 with the compute of batch i;
+    device inputs and outputs are double-buffered, and events order every
+    reuse of a buffer after the work that last touched it.
+    """
+
+    def __init__(self, rt: MoERoundTrip, w_gate, w_up, w_down, compute_stream=None):
+        self.rt = rt
+        self.w = (w_gate, w_up, w_down)
+        dev = rt.device
+        self.comp = compute_stream if compute_stream is not None else torch.cuda.current_stream(dev)
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.x_dev = [torch.empty((rt.T, rt.H), dtype=rt.dtype, device=dev) for _ in range(2)]
+        self.l_dev = [torch.empty((rt.T, rt.E), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.y_dev = [torch.empty((rt.T, rt.H), dtype=rt.dtype, device=dev) for _ in range(2)]
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.in_ready, self.in_free, self.out_ready, self.out_free = ev(), ev(), ev(), ev()
+        self._used = [False, False]
+
+    @staticmethod
+    def _as_dev_dtype(host: torch.Tensor, dev: torch.Tensor) -> torch.Tensor:
+        # bfloat16 data may be held on the host as raw int16 bit patterns
+        return host.view(dev.dtype) if host.dtype != dev.dtype and host.element_size() == dev.element_size() else host
+
+    def run(self, batches):
+        """batches: iterable of (x_host, logits_host, y_host), pinned CPU tensors.
+        Enqueues everything and returns; y_host is valid after the d2h stream syncs."""
+        for i, (xh, lh, yh) in enumerate(batches):
+            b = i & 1
+            if self._used[b]:
+                self.h2d.wait_event(self.in_free[b])   # compute of batch i-2 is done with x/l buffers
+            with torch.cuda.stream(self.h2d):
+                self.x_dev[b].copy_(self._as_dev_dtype(xh, self.x_dev[b]), non_blocking=True)
+                self.l_dev[b].copy_(lh, non_blocking=True)
+                self.in_ready[b].record(self.h2d)
+            self.comp.wait_event(self.in_ready[b])
+            if self._used[b]:
+                self.comp.wait_event(self.out_free[b])  # y of batch i-2 has been copied out
+            self.rt.forward(self.x_dev[b], self.l_dev[b], *self.w, stream=self.comp, y=self.y_dev[b])
+            self.in_free[b].record(self.comp)
+            self.out_ready[b].record(self.comp)
+            self.d2h.wait_event(self.out_ready[b])
+            with torch.cuda.stream(self.d2h):
+                yh.copy_(self.y_dev[b].view(yh.dtype) if yh.dtype != self.y_dev[b].dtype else self.y_dev[b],
+                         non_blocking=True)
+                self.out_free[b].record(self.d2h)
+            self._used[b] = True
+        return self.d2h

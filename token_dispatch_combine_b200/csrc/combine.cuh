@@ -5,20 +5,24 @@
 // original order; "Return multiple expert results to the same token":
 // y(t) = sum_j w_j u_j (e.g. 0.7 u0 + 0.3 u2).
 //
-// One warp per token.  Lanes j < k fetch (row_j, w_j) and broadcast them;
-// then each lane walks 16-byte column chunks, issuing all k row loads before
-// the float32 multiply-adds (fixed order j = 0..k-1) and one rounded store.
+// One warp per (token, slice of 64 16-byte columns).  Lanes j < k fetch
+// (row_j, w_j) and broadcast them; then each lane walks its 16-byte column
+// chunks, issuing all k row loads before the float32 multiply-adds (fixed
+// order j = 0..k-1) and one rounded store.
 #pragma once
 
 #include "common.cuh"
 
 namespace moe {
 
+constexpr int kCombineSlice = 64;  // 16-byte column vectors of a row per warp (2 per lane)
+
 template <typename T, int K>
 __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_disp, const float* __restrict__ topk_w,
                                                       const int32_t* __restrict__ slot_to_row, int T_, int H, int S,
-                                                      T* __restrict__ y) {
-  const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+                                                      int nslices, T* __restrict__ y) {
+  const size_t gw = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5;
+  const int t = (int)(gw / nslices), cs = (int)(gw - (size_t)t * nslices);
   const int lane = (int)lane_id();
   if (t >= T_) return;
   int my_row = -1;
@@ -27,7 +31,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_di
     my_row = __ldg(slot_to_row + (size_t)t * K + lane);
     my_w = __ldg(topk_w + (size_t)t * K + lane);
     if (my_row < 0 || my_row >= S) {
-      if (my_row != -1) flag_error(kErrBadRow);  // -1 marks a slot dispatch dropped
+      if (my_row != -1 && cs == 0) flag_error(kErrBadRow);  // -1 marks a slot dispatch dropped
       my_row = -1;
     }
   }
@@ -41,7 +45,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_di
   constexpr int N = Vec16<T>::N;
   const int nvec = H / N;
   char* dst = reinterpret_cast<char*>(y + (size_t)t * H);
-  for (int i = lane; i < nvec; i += 32) {
+  const int i_end = min(nvec, (cs + 1) * kCombineSlice);
+  for (int i = cs * kCombineSlice + lane; i < i_end; i += 32) {
     uint4 v[K];
 #pragma unroll
     for (int j = 0; j < K; ++j)
@@ -66,12 +71,14 @@ cudaError_t launch_combine(const T* y_disp, const float* topk_w, const int32_t* 
                            T* y, cudaStream_t stream) {
   if (T_ == 0) return cudaSuccess;
   const int threads = 256;
-  const int blocks = (int)(((size_t)T_ * 32 + threads - 1) / threads);
+  const int nvec = H / Vec16<T>::N;
+  const int nslices = (nvec + kCombineSlice - 1) / kCombineSlice;
+  const int blocks = (int)(((size_t)T_ * nslices * 32 + threads - 1) / threads);
   const int S = T_ * k;
   switch (k) {
 #define MOE_COMBINE_CASE(KK) \
   case KK:                   \
-    combine_kernel<T, KK><<<blocks, threads, 0, stream>>>(y_disp, topk_w, slot_to_row, T_, H, S, y); \
+    combine_kernel<T, KK><<<blocks, threads, 0, stream>>>(y_disp, topk_w, slot_to_row, T_, H, S, nslices, y); \
     break;
     MOE_COMBINE_CASE(1)
     MOE_COMBINE_CASE(2)

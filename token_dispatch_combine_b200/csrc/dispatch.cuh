@@ -18,9 +18,10 @@
 //     the earlier warps' counts.  The last CTA to finish (a fence + counter,
 //     no waiting) turns the per-chunk counts into expert offsets, per-chunk
 //     bases, rank counts and source-rank counts.
-//  2. dispatch_scatter_kernel, one warp per token: computes the token's k
-//     rows, writes slot_to_row / row_to_slot, reads the token row once and
-//     stores it to its k rows with 16-byte vector accesses.
+//  2. dispatch_scatter_kernel, one warp per (token, slice of 128 16-byte
+//     columns): computes the token's k rows (the first slice also writes
+//     slot_to_row / row_to_slot), reads its slice of the token row once and
+//     stores it to the k rows with 16-byte vector accesses.
 #pragma once
 
 #include "common.cuh"
@@ -29,7 +30,7 @@ namespace moe {
 
 struct DispatchGeom {
   int T, k, E, R, S;
-  int chunk;    // slots per chunk (= CTA size of kernel 1, a multiple of 32)
+  int chunk;    // slots per chunk (<= the 1024-thread CTA of kernel 1, a multiple of 32)
   int cpr;      // chunks per source rank
   int nchunks;  // R * cpr
   int counts_in_smem;  // the last CTA stages the [nchunks][E] counts in shared memory
@@ -233,8 +234,12 @@ __global__ void __launch_bounds__(1024) dispatch_rank_kernel(
   if (threadIdx.x == 0) *ws.counter = 0u;  // ready for the next call
 }
 
+constexpr int kScatterVecsPerLane = 4;                   // 16-byte vectors in flight per lane
+constexpr int kScatterSlice = 32 * kScatterVecsPerLane;  // 16-byte vectors of a row per warp
+
 template <typename T>
-__global__ void __launch_bounds__(256) dispatch_scatter_kernel(DispatchGeom g, int H, const T* __restrict__ x,
+__global__ void __launch_bounds__(256) dispatch_scatter_kernel(DispatchGeom g, int H, int nslices,
+                                                               const T* __restrict__ x,
                                                                const int32_t* __restrict__ ids, DispatchWs ws,
                                                                const int32_t* __restrict__ expert_offsets,
                                                                T* __restrict__ x_disp,
@@ -246,7 +251,9 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(DispatchGeom g, i
     const int placed = __ldg(expert_offsets + g.E);
     if (gtid < (size_t)(g.S - placed)) row_to_slot[placed + gtid] = -1;
   }
-  const int t = (int)(gtid >> 5);
+  // warp -> (token, column slice of kScatterSlice vectors)
+  const size_t gw = gtid >> 5;
+  const int t = (int)(gw / nslices), cs = (int)(gw - (size_t)t * nslices);
   const int lane = (int)lane_id();
   if (t >= g.T) return;
 
@@ -256,8 +263,10 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(DispatchGeom g, i
     const int e = __ldg(ids + s);
     const int rk = ws.slot_rank[s];
     if (e >= 0 && e < g.E && rk >= 0) my_row = ws.chunk_base[(size_t)chunk_of_slot(g, s) * g.E + e] + rk;
-    slot_to_row[s] = my_row;
-    if (my_row >= 0) row_to_slot[my_row] = s;
+    if (cs == 0) {
+      slot_to_row[s] = my_row;
+      if (my_row >= 0) row_to_slot[my_row] = s;
+    }
   }
   int rows[8];
 #pragma unroll
@@ -266,23 +275,21 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(DispatchGeom g, i
   constexpr int N = Vec16<T>::N;
   const int nvec = H / N;
   const char* src = reinterpret_cast<const char*>(x + (size_t)t * H);
-  constexpr int U = 4;  // 16-byte vectors in flight per lane
-  for (int base = 0; base < nvec; base += 32 * U) {
-    uint4 v[U];
+  const int base = cs * kScatterSlice;
+  uint4 v[kScatterVecsPerLane];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+  for (int u = 0; u < kScatterVecsPerLane; ++u) {
+    const int i = base + u * 32 + lane;
+    if (i < nvec) v[u] = ld_nc_v4(src + (size_t)i * 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= g.k || rows[j] < 0) continue;
+    char* dst = reinterpret_cast<char*>(x_disp + (size_t)rows[j] * H);
+#pragma unroll
+    for (int u = 0; u < kScatterVecsPerLane; ++u) {
       const int i = base + u * 32 + lane;
-      if (i < nvec) v[u] = ld_nc_v4(src + (size_t)i * 16);
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j >= g.k || rows[j] < 0) continue;
-      char* dst = reinterpret_cast<char*>(x_disp + (size_t)rows[j] * H);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = base + u * 32 + lane;
-        if (i < nvec) st_v4(dst + (size_t)i * 16, v[u]);
-      }
+      if (i < nvec) st_v4(dst + (size_t)i * 16, v[u]);
     }
   }
 }
@@ -293,7 +300,7 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
                             int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
                             int32_t* src_expert_counts, cudaStream_t stream) {
   DispatchWs ws = dispatch_ws_carve(workspace, g);
-  const int threads1 = g.chunk;
+  const int threads1 = 1024;  // >= chunk: spare threads speed up the last CTA's scans
   size_t table = (size_t)(threads1 / 32) * g.E;  // warp_counts, later the staged chunk counts
   if (g.counts_in_smem && (size_t)g.nchunks * g.E > table) table = (size_t)g.nchunks * g.E;
   const size_t smem1 = sizeof(int32_t) * (table + g.E + 1);
@@ -307,11 +314,13 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int threads2 = 256;
-  const size_t warps = (size_t)g.T;
+  const int nvec = H / Vec16<T>::N;
+  const int nslices = (nvec + kScatterSlice - 1) / kScatterSlice;
+  const size_t warps = (size_t)g.T * nslices;
   const int blocks2 = (int)((warps * 32 + threads2 - 1) / threads2);
   if (blocks2 > 0)
-    dispatch_scatter_kernel<T><<<blocks2, threads2, 0, stream>>>(g, H, x, ids, ws, expert_offsets, x_disp,
-                                                                 slot_to_row, row_to_slot);
+    dispatch_scatter_kernel<T><<<blocks2, threads2, 0, stream>>>(g, H, nslices, x, ids, ws, expert_offsets,
+                                                                 x_disp, slot_to_row, row_to_slot);
   return cudaGetLastError();
 }
 

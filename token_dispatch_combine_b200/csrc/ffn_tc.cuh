@@ -46,7 +46,7 @@
 //  MOE_TC_HINT_A / MOE_TC_HINT_B: L2 eviction priority of the TMA loads of the
 //    activation and weight tiles (0 normal, 1 evict-first, 2 evict-last).
 #ifndef MOE_TC_GROUP_M
-#define MOE_TC_GROUP_M 0
+#define MOE_TC_GROUP_M 16
 #endif
 #ifndef MOE_TC_HINT_A
 #define MOE_TC_HINT_A 0
