@@ -21,6 +21,8 @@ template <typename T, int K>
 __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_disp, const float* __restrict__ topk_w,
                                                       const int32_t* __restrict__ slot_to_row, int T_, int H, int S,
                                                       int nslices, T* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const size_t gw = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5;
   const int t = (int)(gw / nslices), cs = (int)(gw - (size_t)t * nslices);
   const int lane = (int)lane_id();
@@ -75,10 +77,12 @@ cudaError_t launch_combine(const T* y_disp, const float* topk_w, const int32_t* 
   const int nslices = (nvec + kCombineSlice - 1) / kCombineSlice;
   const int blocks = (int)(((size_t)T_ * nslices * 32 + threads - 1) / threads);
   const int S = T_ * k;
+  cudaError_t err = cudaSuccess;
   switch (k) {
 #define MOE_COMBINE_CASE(KK) \
   case KK:                   \
-    combine_kernel<T, KK><<<blocks, threads, 0, stream>>>(y_disp, topk_w, slot_to_row, T_, H, S, nslices, y); \
+    err = launch_pdl(combine_kernel<T, KK>, blocks, threads, 0, stream, y_disp, topk_w, slot_to_row, T_, H, S, \
+                     nslices, y);                                                                                \
     break;
     MOE_COMBINE_CASE(1)
     MOE_COMBINE_CASE(2)
@@ -92,7 +96,7 @@ cudaError_t launch_combine(const T* y_disp, const float* topk_w, const int32_t* 
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe_b200.h"
 
 namespace moe {
@@ -22,6 +24,33 @@ __device__ uint32_t g_error_word;
 __device__ __forceinline__ void flag_error(uint32_t bits) { atomicOr(&g_error_word, bits); }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
+
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with programmatic stream serialisation, so it may start while the previous
+// kernel in the stream is still finishing.  pdl_wait() blocks until that
+// kernel has completed and its memory is visible; no global memory that a
+// predecessor touches may be read or written before it.  pdl_trigger() lets
+// the next kernel in the stream begin launching (it still waits in its own
+// pdl_wait() for this one to complete).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch with programmatic stream serialisation allowed (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

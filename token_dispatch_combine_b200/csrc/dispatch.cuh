@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(1024) dispatch_rank_kernel(
   int32_t* scan = smem_i32 + table;  // [E + 1]
   __shared__ int s_is_last;
 
+  pdl_wait();
+  pdl_trigger();
   const int c = blockIdx.x;
   int s0, s1;
   chunk_slot_range(g, c, s0, s1);
@@ -245,6 +247,8 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(DispatchGeom g, i
                                                                T* __restrict__ x_disp,
                                                                int32_t* __restrict__ slot_to_row,
                                                                int32_t* __restrict__ row_to_slot) {
+  pdl_wait();
+  pdl_trigger();
   const size_t gtid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   // rows past the last placed row (only when ids were dropped) get row_to_slot = -1
   {
@@ -309,18 +313,20 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
                                            (int)smem1);
     if (err != cudaSuccess) return err;
   }
-  dispatch_rank_kernel<<<g.nchunks, threads1, smem1, stream>>>(g, ids, ws, expert_counts, expert_offsets,
-                                                               rank_counts, rank_offsets, src_expert_counts);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(dispatch_rank_kernel, g.nchunks, threads1, smem1, stream, g, ids, ws, expert_counts,
+                               expert_offsets, rank_counts, rank_offsets, src_expert_counts);
+  if (err == cudaSuccess) err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int threads2 = 256;
   const int nvec = H / Vec16<T>::N;
   const int nslices = (nvec + kScatterSlice - 1) / kScatterSlice;
   const size_t warps = (size_t)g.T * nslices;
   const int blocks2 = (int)((warps * 32 + threads2 - 1) / threads2);
-  if (blocks2 > 0)
-    dispatch_scatter_kernel<T><<<blocks2, threads2, 0, stream>>>(g, H, nslices, x, ids, ws, expert_offsets,
-                                                                 x_disp, slot_to_row, row_to_slot);
+  if (blocks2 > 0) {
+    err = launch_pdl(dispatch_scatter_kernel<T>, blocks2, threads2, 0, stream, g, H, nslices, x, ids, ws,
+                     expert_offsets, x_disp, slot_to_row, row_to_slot);
+    if (err != cudaSuccess) return err;
+  }
   return cudaGetLastError();
 }
 

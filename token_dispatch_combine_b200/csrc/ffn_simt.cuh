@@ -40,6 +40,8 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A, 
   __shared__ float Bs0[BK][BN];
   __shared__ float Bs1[GATEUP ? BK : 1][GATEUP ? BN : 1];
 
+  pdl_wait();
+  pdl_trigger();
   // map blockIdx.x -> (expert, m-tile)
   int e = -1, row0 = 0, row_end = 0;
   {
@@ -120,8 +122,8 @@ cudaError_t launch_ffn_simt_gate_up(const T* x_disp, const T* wg, const T* wu, c
   const int max_mtiles = (S + 63) / 64 + E;  // bound on sum_e ceil(count_e / 64)
   if (S == 0) return cudaSuccess;
   dim3 grid(max_mtiles, (I + 63) / 64);
-  ffn_simt_kernel<T, true><<<grid, 256, 0, stream>>>(x_disp, wg, wu, off, E, H, I, S, h);
-  return cudaGetLastError();
+  cudaError_t err = launch_pdl(ffn_simt_kernel<T, true>, grid, 256, 0, stream, x_disp, wg, wu, off, E, H, I, S, h);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 template <typename T>
@@ -130,8 +132,9 @@ cudaError_t launch_ffn_simt_down(const T* h, const T* wd, const int32_t* off, in
   const int max_mtiles = (S + 63) / 64 + E;
   if (S == 0) return cudaSuccess;
   dim3 grid(max_mtiles, (H + 63) / 64);
-  ffn_simt_kernel<T, false><<<grid, 256, 0, stream>>>(h, wd, nullptr, off, E, I, H, S, y);
-  return cudaGetLastError();
+  cudaError_t err = launch_pdl(ffn_simt_kernel<T, false>, grid, 256, 0, stream, h, wd, (const T*)nullptr, off, E, I,
+                               H, S, y);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -277,6 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (GATEUP) prefetch_tmap(&tmap_b1);
   }
   if (warp == 1) tmem_alloc(smem_u32(s_tmem), kTmemCols);
+  // Everything above touches only this CTA's shared memory and TMEM; from here
+  // on the kernel reads what earlier kernels wrote.
+  pdl_wait();
+  pdl_trigger();
   if (warp == 2) {
     // clamped segment starts and per-expert m-tile prefix sums (warp scan)
     const int E = p.E;
@@ -596,8 +600,8 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUten
   const long long max_tiles = ((long long)(p.S + BM - 1) / BM + p.E) * p.ntn;
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
-  kern<<<grid, kThreads, smem, stream>>>(ta, tb0, tb1, p);
-  return cudaGetLastError();
+  cudaError_t err = launch_pdl(kern, grid, kThreads, smem, stream, ta, tb0, tb1, p);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 // h = SiLU(x_disp Wg) * (x_disp Wu), 128-column h tiles (MMA N = 256)

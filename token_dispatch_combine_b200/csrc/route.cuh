@@ -28,6 +28,8 @@ template <int VPL>  // logits per lane: ceil(E / 32)
 __global__ void __launch_bounds__(256) route_topk_softmax_kernel(const float* __restrict__ logits, int T, int E,
                                                                  int k, int32_t* __restrict__ topk_ids,
                                                                  float* __restrict__ topk_w) {
+  pdl_wait();
+  pdl_trigger();
   const int t = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = (int)lane_id();
   if (t >= T) return;  // whole warp exits together
@@ -81,9 +83,10 @@ inline cudaError_t launch_route(const float* logits, int T, int E, int k, int32_
   const int threads = 256;
   const int blocks = (int)(((size_t)T * 32 + threads - 1) / threads);
   const int vpl = (E + 31) / 32;
+  cudaError_t err = cudaSuccess;
 #define MOE_ROUTE_CASE(V)                                                                  \
   case V:                                                                                  \
-    route_topk_softmax_kernel<V><<<blocks, threads, 0, stream>>>(logits, T, E, k, ids, w); \
+    err = launch_pdl(route_topk_softmax_kernel<V>, blocks, threads, 0, stream, logits, T, E, k, ids, w); \
     break;
   switch (vpl <= 1 ? 1 : vpl <= 2 ? 2 : vpl <= 4 ? 4 : vpl <= 8 ? 8 : vpl <= 16 ? 16 : 32) {
     MOE_ROUTE_CASE(1)
@@ -94,7 +97,7 @@ inline cudaError_t launch_route(const float* logits, int T, int E, int k, int32_
     MOE_ROUTE_CASE(32)
   }
 #undef MOE_ROUTE_CASE
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe
