@@ -54,6 +54,10 @@
 #ifndef MOE_TC_HINT_B
 #define MOE_TC_HINT_B 0
 #endif
+//  MOE_TC_DOWN_BN: force the down-projection n-tile width (0 = chosen from H).
+#ifndef MOE_TC_DOWN_BN
+#define MOE_TC_DOWN_BN 0
+#endif
 
 namespace moe {
 namespace tc {
@@ -621,22 +625,25 @@ inline cudaError_t launch_down(const void* h, const void* wd, const int32_t* off
   if (S == 0) return cudaSuccess;
   CUtensorMap ta, tb;
   if (!make_tmap_act(&ta, h, S, I) || !make_tmap_weight(&tb, wd, E, I, H)) return cudaErrorInvalidValue;
-  const int cands[4] = {256, 240, 192, 128};
+  // n-tile width: UMMA N that is a whole number of 64-column boxes runs best
+  // (measured: N = 240 is slower than N = 256 even counting 256's padding), so
+  // pick among 256 / 192 / 128 by padded width times a per-width cost.
+  const int cands[3] = {256, 192, 128};
+  const double cost[3] = {1.0, 1.08, 1.3};
   int best = 256;
-  long long best_pad = -1;
-  for (int bn : cands) {
-    const long long pad = (long long)((H + bn - 1) / bn) * bn;
-    if (best_pad < 0 || pad < best_pad) {
-      best_pad = pad;
-      best = bn;
+  double best_cost = -1.0;
+  for (int i = 0; i < 3; ++i) {
+    const double c = (double)((H + cands[i] - 1) / cands[i]) * cands[i] * cost[i];
+    if (best_cost < 0 || c < best_cost) {
+      best_cost = c;
+      best = cands[i];
     }
   }
+  if (MOE_TC_DOWN_BN > 0) best = MOE_TC_DOWN_BN;
   Params p{off, E, S, I, H, (H + best - 1) / best, reinterpret_cast<__nv_bfloat16*>(y)};
   switch (best) {
     case 256:
       return launch_tc<false, 256, 4>(ta, tb, tb, p, stream);
-    case 240:
-      return launch_tc<false, 240, 4>(ta, tb, tb, p, stream);
     case 192:
       return launch_tc<false, 192, 5>(ta, tb, tb, p, stream);
     default:
