@@ -8,35 +8,43 @@
 // "Expert Parallelism (EP)", "Limitations" 3-4: rank r owns experts
 // [r*E/R, (r+1)*E/R), so the expert-major row order is rank-major.
 //
-// Two launches:
-//  1. dispatch_rank_kernel, one CTA per chunk of slots.  Chunks never straddle
-//     a source rank (token t's source rank is t*R/T), so per-(source rank,
-//     expert) counts are sums of whole chunks.  Each slot gets its stable rank
-//     among same-expert slots of its chunk without atomics:
-//     __match_any_sync groups a warp's lanes by expert, popc of the lower
-//     peers gives the in-warp rank, and a per-expert scan over the warps adds
-//     the earlier warps' counts.  The last CTA to finish (a fence + counter,
-//     no waiting) turns the per-chunk counts into expert offsets, per-chunk
-//     bases, rank counts and source-rank counts.
-//  2. dispatch_scatter_kernel, one warp per (token, slice of 128 16-byte
-//     columns): computes the token's k rows (the first slice also writes
-//     slot_to_row / row_to_slot), reads its slice of the token row once and
-//     stores it to the k rows with 16-byte vector accesses.
+// One cooperative launch (every CTA resident at once), three phases split by
+// two bounded grid barriers:
+//  1. per chunk of <= 512 slots (chunks never straddle a source rank, token
+//     t's source rank being t*R/T): each slot's stable rank among the
+//     same-expert slots of its chunk, without atomics -- __match_any_sync
+//     groups a warp's lanes by expert, popc of the lower peers gives the
+//     in-warp rank, a per-expert scan over the CTA's warps adds the earlier
+//     warps' counts -- and the chunk's per-expert counts;
+//  2. one warp per expert scans that expert's counts over the chunks (warp
+//     prefix sums, 32 chunks per round) into per-chunk bases and a total;
+//     after the second barrier every CTA scans the E totals into expert
+//     offsets in shared memory;
+//  3. one warp per (token, slice of 128 16-byte columns) computes the token's
+//     k rows (offset + chunk base + in-chunk rank), writes the permutation
+//     (first slice only), and copies its slice of the token row to the k rows
+//     with 16-byte vector accesses.  Each warp loads its first slice of x
+//     before phase 1, so that read overlaps the counting and the barriers.
+// A barrier that does not complete within 1 s sets the timeout bit of the
+// device error word; the kernel then returns without writing the rows.
 #pragma once
 
 #include "common.cuh"
 
 namespace moe {
 
+constexpr int kDispatchThreads = 512;
+constexpr int kDispatchWarps = kDispatchThreads / 32;
+constexpr int kScatterVecsPerLane = 4;                   // 16-byte vectors in flight per lane
+constexpr int kScatterSlice = 32 * kScatterVecsPerLane;  // 16-byte vectors of a row per warp item
+constexpr uint64_t kGridBarrierLimitNs = 1000000000ull;   // 1 s
+
 struct DispatchGeom {
   int T, k, E, R, S;
-  int chunk;    // slots per chunk (<= the 1024-thread CTA of kernel 1, a multiple of 32)
+  int chunk;    // slots per chunk (<= kDispatchThreads, a multiple of 32)
   int cpr;      // chunks per source rank
   int nchunks;  // R * cpr
-  int counts_in_smem;  // the last CTA stages the [nchunks][E] counts in shared memory
 };
-
-constexpr size_t kDispatchCountsSmemMax = 96 * 1024;  // bytes of [nchunks][E] counts staged by the last CTA
 
 // First token of source rank r: ceil(r*T/R), so that t*R/T == r on [lo(r), lo(r+1)).
 __host__ __device__ __forceinline__ int src_rank_first_token(int r, int T, int R) {
@@ -53,36 +61,40 @@ inline DispatchGeom make_dispatch_geom(int T, int k, int E, int R) {
   const int max_tok = (T + R - 1) / R;  // largest source-rank range
   const int max_slots = max_tok * k;
   int ch = ((max_slots + 31) / 32) * 32;
-  if (ch > 1024) ch = 1024;
+  if (ch > kDispatchThreads) ch = kDispatchThreads;
   if (ch < 32) ch = 32;
   g.chunk = ch;
   g.cpr = (max_slots + ch - 1) / ch;
   if (g.cpr < 1) g.cpr = 1;
   g.nchunks = R * g.cpr;
-  g.counts_in_smem = (size_t)g.nchunks * E * sizeof(int32_t) <= kDispatchCountsSmemMax;
   return g;
 }
 
-// Workspace layout (bytes): [0,256) control word; chunk_counts[nchunks][E];
-// chunk_base[nchunks][E]; slot_rank[S].
+// Workspace layout (bytes): [0,256) control words (grid-barrier arrival count
+// at 64, generation at 128); chunk_counts[nchunks][E]; chunk_base[nchunks][E]
+// (relative to the expert's offset); slot_rank[S]; totals[E].
 struct DispatchWs {
-  uint32_t* counter;
+  uint32_t* bar_count;
+  uint32_t* bar_gen;
   int32_t* chunk_counts;
   int32_t* chunk_base;
   int32_t* slot_rank;
+  int32_t* totals;
 };
 
 inline size_t dispatch_ws_bytes(const DispatchGeom& g) {
-  return 256 + sizeof(int32_t) * ((size_t)2 * g.nchunks * g.E + (size_t)g.S);
+  return 256 + sizeof(int32_t) * ((size_t)2 * g.nchunks * g.E + (size_t)g.S + (size_t)g.E);
 }
 
 inline DispatchWs dispatch_ws_carve(void* base, const DispatchGeom& g) {
   char* p = (char*)base;
   DispatchWs w;
-  w.counter = (uint32_t*)p;
+  w.bar_count = (uint32_t*)(p + 64);
+  w.bar_gen = (uint32_t*)(p + 128);
   w.chunk_counts = (int32_t*)(p + 256);
   w.chunk_base = w.chunk_counts + (size_t)g.nchunks * g.E;
   w.slot_rank = w.chunk_base + (size_t)g.nchunks * g.E;
+  w.totals = w.slot_rank + (size_t)g.S;
   return w;
 }
 
@@ -102,198 +114,215 @@ __device__ __forceinline__ int chunk_of_slot(const DispatchGeom& g, int s) {
   return r * g.cpr + (s - lo) / g.chunk;
 }
 
-// Dynamic shared memory: warp_counts[nwarps][E] int32, then E + 1 ints for the scan.
-__global__ void __launch_bounds__(1024) dispatch_rank_kernel(
-    DispatchGeom g, const int32_t* __restrict__ ids, DispatchWs ws, int32_t* __restrict__ expert_counts,
-    int32_t* __restrict__ expert_offsets, int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets,
-    int32_t* __restrict__ src_expert_counts) {
-  extern __shared__ int32_t smem_i32[];
-  const int nwarps = blockDim.x >> 5;
-  const int warp = threadIdx.x >> 5, lane = (int)lane_id();
-  int32_t* warp_counts = smem_i32;  // [nwarps][E]
-  size_t table = (size_t)nwarps * g.E;
-  if (g.counts_in_smem && (size_t)g.nchunks * g.E > table) table = (size_t)g.nchunks * g.E;
-  int32_t* scan = smem_i32 + table;  // [E + 1]
-  __shared__ int s_is_last;
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
+// Grid-wide barrier for a cooperative launch.  Thread 0 of each CTA reads the
+// generation, arrives on the counter; the last arrival resets the counter and
+// bumps the generation; the others wait (bounded) for the bump.  Returns
+// false, with the timeout bit set, if the wait gave up.
+__device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t gen = ld_acquire_u32(ws.bar_gen);
+    __threadfence();
+    const uint32_t arrived = atomicAdd(ws.bar_count, 1u);
+    if (arrived == gridDim.x - 1) {
+      atomicExch(ws.bar_count, 0u);
+      __threadfence();
+      atomicAdd(ws.bar_gen, 1u);
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_u32(ws.bar_gen) == gen) {
+        if (globaltimer_ns() - t0 > kGridBarrierLimitNs) {
+          flag_error(kErrTimeout);
+          *s_ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+// Dynamic shared memory: warp_counts[kDispatchWarps][E] int32, then offs[E + 1].
+template <typename T>
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
+    DispatchGeom g, int H, int nslices, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
+    T* __restrict__ x_disp, int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
+    int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_to_row,
+    int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
+  extern __shared__ int32_t smem_i32[];
+  int32_t* warp_counts = smem_i32;                          // [kDispatchWarps][E]
+  int32_t* offs = smem_i32 + (size_t)kDispatchWarps * g.E;  // [E + 1]
+  __shared__ int s_ok;
   pdl_wait();
   pdl_trigger();
-  const int c = blockIdx.x;
-  int s0, s1;
-  chunk_slot_range(g, c, s0, s1);
+  const int warp = threadIdx.x >> 5, lane = (int)lane_id();
+  const size_t gwarp = (size_t)blockIdx.x * kDispatchWarps + warp;
+  const size_t nwarps_grid = (size_t)gridDim.x * kDispatchWarps;
+  const size_t gtid = (size_t)blockIdx.x * kDispatchThreads + threadIdx.x;
+  const size_t nthreads_grid = (size_t)gridDim.x * kDispatchThreads;
+  if (threadIdx.x == 0) s_ok = 1;
 
-  for (int i = threadIdx.x; i < nwarps * g.E; i += blockDim.x) warp_counts[i] = 0;
-  __syncthreads();
-
-  const int s = s0 + (int)threadIdx.x;
-  int e = -2;  // -2: no slot; -1: bad id
-  if (s < s1) {
-    e = __ldg(ids + s);
-    if (e < 0 || e >= g.E) {
-      flag_error(kErrBadId);
-      e = -1;
+  // ---- prefetch this warp's first slice of x (it does not depend on the counts)
+  constexpr int N = Vec16<T>::N;
+  const int nvec = H / N;
+  const size_t nitems = (size_t)g.T * nslices;
+  uint4 pre[kScatterVecsPerLane];
+  if (gwarp < nitems) {
+    const int t = (int)(gwarp / nslices), cs = (int)(gwarp - (size_t)t * nslices);
+    const char* src = reinterpret_cast<const char*>(x + (size_t)t * H);
+#pragma unroll
+    for (int u = 0; u < kScatterVecsPerLane; ++u) {
+      const int i = cs * kScatterSlice + u * 32 + lane;
+      if (i < nvec) pre[u] = ld_nc_v4(src + (size_t)i * 16);
     }
   }
-  const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
-  const int rank_in_warp = __popc(peers & ((1u << lane) - 1u));
-  if (e >= 0 && lane == __ffs(peers) - 1) warp_counts[warp * g.E + e] = __popc(peers);
-  __syncthreads();
-  // exclusive scan over warps, per expert; totals are this chunk's counts
-  for (int x = threadIdx.x; x < g.E; x += blockDim.x) {
-    int run = 0;
-    for (int w = 0; w < nwarps; ++w) {
-      const int v = warp_counts[w * g.E + x];
-      warp_counts[w * g.E + x] = run;
-      run += v;
-    }
-    ws.chunk_counts[(size_t)c * g.E + x] = run;
-  }
-  __syncthreads();
-  if (s < s1) ws.slot_rank[s] = (e >= 0) ? warp_counts[warp * g.E + e] + rank_in_warp : -1;
 
-  // ---- last CTA: global scans (no CTA ever waits for another) ----
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_is_last = (atomicAdd(ws.counter, 1u) == (uint32_t)(g.nchunks - 1));
-  __syncthreads();
-  if (!s_is_last) return;
-  __threadfence();
-
-  // The per-chunk counts come back through L2; every read below is issued
-  // independently of the running sums so that many are in flight at once.
-  const int nce = g.nchunks * g.E;
-  int32_t* cnt = smem_i32;  // warp_counts is dead here: reuse it for the [nchunks][E] counts
-  if (g.counts_in_smem) {
-#pragma unroll 4
-    for (int i = threadIdx.x; i < nce; i += blockDim.x) cnt[i] = __ldcg(ws.chunk_counts + i);
+  // ---- phase 1: per-chunk stable ranks and counts
+  for (int c = blockIdx.x; c < g.nchunks; c += gridDim.x) {
+    int s0, s1;
+    chunk_slot_range(g, c, s0, s1);
+    for (int i = threadIdx.x; i < kDispatchWarps * g.E; i += kDispatchThreads) warp_counts[i] = 0;
     __syncthreads();
-  }
-  auto count_at = [&](int cc, int x) {
-    return g.counts_in_smem ? cnt[cc * g.E + x] : __ldcg(ws.chunk_counts + (size_t)cc * g.E + x);
-  };
-  // 1. per-expert totals
-  for (int x = threadIdx.x; x < g.E; x += blockDim.x) {
-    int run = 0;
-    for (int c0 = 0; c0 < g.nchunks; c0 += 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = (c0 + u < g.nchunks) ? count_at(c0 + u, x) : 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) run += v[u];
+    const int s = s0 + (int)threadIdx.x;
+    int e = -2;  // -2: no slot; -1: bad id
+    if (s < s1) {
+      e = __ldg(ids + s);
+      if (e < 0 || e >= g.E) {
+        flag_error(kErrBadId);
+        e = -1;
+      }
     }
-    scan[x] = run;
-    expert_counts[x] = run;
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank_in_warp = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && lane == __ffs(peers) - 1) warp_counts[warp * g.E + e] = __popc(peers);
+    __syncthreads();
+    for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) {  // exclusive scan over warps, per expert
+      int run = 0;
+#pragma unroll
+      for (int w = 0; w < kDispatchWarps; ++w) {
+        const int v = warp_counts[w * g.E + xx];
+        warp_counts[w * g.E + xx] = run;
+        run += v;
+      }
+      ws.chunk_counts[(size_t)c * g.E + xx] = run;
+    }
+    __syncthreads();
+    if (s < s1) ws.slot_rank[s] = (e >= 0) ? warp_counts[warp * g.E + e] + rank_in_warp : -1;
+    __syncthreads();  // warp_counts is reused by the next chunk
   }
-  __syncthreads();
-  // 2. exclusive scan over experts (warp 0, 32 at a time)
-  if (warp == 0) {
+  if (!grid_barrier(ws, &s_ok)) return;
+
+  // ---- phase 2a: one warp per expert, prefix over chunks
+  for (size_t e = gwarp; e < (size_t)g.E; e += nwarps_grid) {
     int carry = 0;
-    for (int base = 0; base < g.E; base += 32) {
-      const int v = (base + lane < g.E) ? scan[base + lane] : 0;
+    for (int base = 0; base < g.nchunks; base += 32) {
+      const int c = base + lane;
+      const int v = (c < g.nchunks) ? __ldcg(ws.chunk_counts + (size_t)c * g.E + e) : 0;
       int incl = v;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
         const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
         if (lane >= d) incl += y;
       }
-      if (base + lane < g.E) scan[base + lane] = carry + incl - v;
+      if (c < g.nchunks) ws.chunk_base[(size_t)c * g.E + e] = carry + incl - v;
       carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
-    if (lane == 0) scan[g.E] = carry;
+    if (lane == 0) {
+      ws.totals[e] = carry;
+      expert_counts[e] = carry;
+    }
+  }
+  if (!grid_barrier(ws, &s_ok)) return;
+
+  // ---- phase 2b: expert offsets (every CTA, in shared memory)
+  for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) offs[xx] = __ldcg(ws.totals + xx);
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < g.E; base += 32) {
+      const int v = (base + lane < g.E) ? offs[base + lane] : 0;
+      int incl = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += y;
+      }
+      if (base + lane < g.E) offs[base + lane] = carry + incl - v;
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) offs[g.E] = carry;
   }
   __syncthreads();
-  // 3. chunk bases = expert offset + counts of the same expert in earlier chunks
-  for (int x = threadIdx.x; x < g.E; x += blockDim.x) {
-    int run = scan[x];
-    for (int c0 = 0; c0 < g.nchunks; c0 += 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = (c0 + u < g.nchunks) ? count_at(c0 + u, x) : 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (c0 + u < g.nchunks) {
-          ws.chunk_base[(size_t)(c0 + u) * g.E + x] = run;
-          run += v[u];
-        }
+  const int placed = offs[g.E];
+  if (blockIdx.x == 0) {
+    for (int xx = threadIdx.x; xx <= g.E; xx += kDispatchThreads) expert_offsets[xx] = offs[xx];
+    const int EL = g.E / g.R;
+    for (int r = threadIdx.x; r < g.R; r += kDispatchThreads) {
+      rank_counts[r] = offs[(r + 1) * EL] - offs[r * EL];
+      rank_offsets[r] = offs[r * EL];
+    }
+    if (threadIdx.x == 0) rank_offsets[g.R] = placed;
+  }
+  if (src_expert_counts) {  // a source rank's chunks are contiguous: differences of the chunk bases
+    for (size_t i = gtid; i < (size_t)g.R * g.E; i += nthreads_grid) {
+      const int r = (int)(i / g.E), xx = (int)(i - (size_t)r * g.E);
+      const int lo = __ldcg(ws.chunk_base + (size_t)(r * g.cpr) * g.E + xx);
+      const int hi = (r + 1 < g.R) ? __ldcg(ws.chunk_base + (size_t)((r + 1) * g.cpr) * g.E + xx)
+                                   : offs[xx + 1] - offs[xx];
+      src_expert_counts[i] = hi - lo;
+    }
+  }
+  // rows past the last placed row (only when ids were dropped) get row_to_slot = -1
+  for (size_t i = gtid; i < (size_t)(g.S - placed); i += nthreads_grid) row_to_slot[placed + i] = -1;
+
+  // ---- phase 3: rows
+  for (size_t item = gwarp; item < nitems; item += nwarps_grid) {
+    const int t = (int)(item / nslices), cs = (int)(item - (size_t)t * nslices);
+    int my_row = -1;
+    if (lane < g.k) {
+      const int s = t * g.k + lane;
+      const int e = __ldg(ids + s);
+      const int rk = __ldcg(ws.slot_rank + s);
+      if (e >= 0 && e < g.E && rk >= 0)
+        my_row = offs[e] + __ldcg(ws.chunk_base + (size_t)chunk_of_slot(g, s) * g.E + e) + rk;
+      if (cs == 0) {
+        slot_to_row[s] = my_row;
+        if (my_row >= 0) row_to_slot[my_row] = s;
       }
     }
-  }
-  for (int x = threadIdx.x; x <= g.E; x += blockDim.x) expert_offsets[x] = scan[x];
-  const int EL = g.E / g.R;
-  for (int r = threadIdx.x; r < g.R; r += blockDim.x) {
-    rank_counts[r] = scan[(r + 1) * EL] - scan[r * EL];
-    rank_offsets[r] = scan[r * EL];
-  }
-  if (threadIdx.x == 0) rank_offsets[g.R] = scan[g.E];
-  if (src_expert_counts) {
-    for (int i = threadIdx.x; i < g.R * g.E; i += blockDim.x) {
-      const int r = i / g.E, x = i - r * g.E;
-      int sum = 0;
-      for (int ci = 0; ci < g.cpr; ++ci) sum += count_at(r * g.cpr + ci, x);
-      src_expert_counts[i] = sum;
+    int rows[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xFFFFFFFFu, my_row, j);
+    uint4 v[kScatterVecsPerLane];
+    if (item == gwarp) {
+#pragma unroll
+      for (int u = 0; u < kScatterVecsPerLane; ++u) v[u] = pre[u];
+    } else {
+      const char* src = reinterpret_cast<const char*>(x + (size_t)t * H);
+#pragma unroll
+      for (int u = 0; u < kScatterVecsPerLane; ++u) {
+        const int i = cs * kScatterSlice + u * 32 + lane;
+        if (i < nvec) v[u] = ld_nc_v4(src + (size_t)i * 16);
+      }
     }
-  }
-  if (threadIdx.x == 0) *ws.counter = 0u;  // ready for the next call
-}
-
-constexpr int kScatterVecsPerLane = 4;                   // 16-byte vectors in flight per lane
-constexpr int kScatterSlice = 32 * kScatterVecsPerLane;  // 16-byte vectors of a row per warp
-
-template <typename T>
-__global__ void __launch_bounds__(256) dispatch_scatter_kernel(DispatchGeom g, int H, int nslices,
-                                                               const T* __restrict__ x,
-                                                               const int32_t* __restrict__ ids, DispatchWs ws,
-                                                               const int32_t* __restrict__ expert_offsets,
-                                                               T* __restrict__ x_disp,
-                                                               int32_t* __restrict__ slot_to_row,
-                                                               int32_t* __restrict__ row_to_slot) {
-  pdl_wait();
-  pdl_trigger();
-  const size_t gtid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
-  // rows past the last placed row (only when ids were dropped) get row_to_slot = -1
-  {
-    const int placed = __ldg(expert_offsets + g.E);
-    if (gtid < (size_t)(g.S - placed)) row_to_slot[placed + gtid] = -1;
-  }
-  // warp -> (token, column slice of kScatterSlice vectors)
-  const size_t gw = gtid >> 5;
-  const int t = (int)(gw / nslices), cs = (int)(gw - (size_t)t * nslices);
-  const int lane = (int)lane_id();
-  if (t >= g.T) return;
-
-  int my_row = -1;
-  if (lane < g.k) {
-    const int s = t * g.k + lane;
-    const int e = __ldg(ids + s);
-    const int rk = ws.slot_rank[s];
-    if (e >= 0 && e < g.E && rk >= 0) my_row = ws.chunk_base[(size_t)chunk_of_slot(g, s) * g.E + e] + rk;
-    if (cs == 0) {
-      slot_to_row[s] = my_row;
-      if (my_row >= 0) row_to_slot[my_row] = s;
-    }
-  }
-  int rows[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xFFFFFFFFu, my_row, j);
-
-  constexpr int N = Vec16<T>::N;
-  const int nvec = H / N;
-  const char* src = reinterpret_cast<const char*>(x + (size_t)t * H);
-  const int base = cs * kScatterSlice;
-  uint4 v[kScatterVecsPerLane];
+    for (int j = 0; j < 8; ++j) {
+      if (j >= g.k || rows[j] < 0) continue;
+      char* dst = reinterpret_cast<char*>(x_disp + (size_t)rows[j] * H);
 #pragma unroll
-  for (int u = 0; u < kScatterVecsPerLane; ++u) {
-    const int i = base + u * 32 + lane;
-    if (i < nvec) v[u] = ld_nc_v4(src + (size_t)i * 16);
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j >= g.k || rows[j] < 0) continue;
-    char* dst = reinterpret_cast<char*>(x_disp + (size_t)rows[j] * H);
-#pragma unroll
-    for (int u = 0; u < kScatterVecsPerLane; ++u) {
-      const int i = base + u * 32 + lane;
-      if (i < nvec) st_v4(dst + (size_t)i * 16, v[u]);
+      for (int u = 0; u < kScatterVecsPerLane; ++u) {
+        const int i = cs * kScatterSlice + u * 32 + lane;
+        if (i < nvec) st_v4(dst + (size_t)i * 16, v[u]);
+      }
     }
   }
 }
@@ -304,30 +333,46 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
                             int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
                             int32_t* src_expert_counts, cudaStream_t stream) {
   DispatchWs ws = dispatch_ws_carve(workspace, g);
-  const int threads1 = 1024;  // >= chunk: spare threads speed up the last CTA's scans
-  size_t table = (size_t)(threads1 / 32) * g.E;  // warp_counts, later the staged chunk counts
-  if (g.counts_in_smem && (size_t)g.nchunks * g.E > table) table = (size_t)g.nchunks * g.E;
-  const size_t smem1 = sizeof(int32_t) * (table + g.E + 1);
-  if (smem1 > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(dispatch_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem1);
-    if (err != cudaSuccess) return err;
-  }
-  cudaError_t err = launch_pdl(dispatch_rank_kernel, g.nchunks, threads1, smem1, stream, g, ids, ws, expert_counts,
-                               expert_offsets, rank_counts, rank_offsets, src_expert_counts);
-  if (err == cudaSuccess) err = cudaGetLastError();
+  auto kern = dispatch_kernel<T>;
+  const size_t smem = sizeof(int32_t) * ((size_t)kDispatchWarps * g.E + g.E + 1);
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  const int threads2 = 256;
+  static int attr_dev = -1;
+  if (attr_dev != dev) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(sizeof(int32_t) * ((size_t)kDispatchWarps * 1024 + 1025)));
+    if (err != cudaSuccess) return err;
+    attr_dev = dev;
+  }
+  // Co-residency bound of the cooperative grid for this shared-memory size.
+  int per_sm = 0, sms = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDispatchThreads, smem);
+  if (err != cudaSuccess) return err;
+  err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (err != cudaSuccess) return err;
+  const long long cap = (long long)per_sm * sms;
+  if (cap < 1) return cudaErrorCooperativeLaunchTooLarge;
   const int nvec = H / Vec16<T>::N;
   const int nslices = (nvec + kScatterSlice - 1) / kScatterSlice;
-  const size_t warps = (size_t)g.T * nslices;
-  const int blocks2 = (int)((warps * 32 + threads2 - 1) / threads2);
-  if (blocks2 > 0) {
-    err = launch_pdl(dispatch_scatter_kernel<T>, blocks2, threads2, 0, stream, g, H, nslices, x, ids, ws,
-                     expert_offsets, x_disp, slot_to_row, row_to_slot);
-    if (err != cudaSuccess) return err;
-  }
-  return cudaGetLastError();
+  const long long item_ctas = ((long long)g.T * nslices + kDispatchWarps - 1) / kDispatchWarps;
+  long long want = item_ctas > g.nchunks ? item_ctas : (long long)g.nchunks;
+  if (want < 1) want = 1;
+  const int grid = (int)(want < cap ? want : cap);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDispatchThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, x, ids, ws, x_disp, expert_counts, expert_offsets, rank_counts,
+                           rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe
