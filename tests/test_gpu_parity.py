@@ -176,3 +176,31 @@ def test_host_pipeline_matches_forward():
     torch.cuda.synchronize()
     for (_, _, yh), y in zip(batches, want):
         assert torch.equal(yh, y.view(torch.int16).cpu())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_graph_replay_matches_forward(dtype):
+    """The whole round trip captured in a CUDA graph gives the eager result, and a
+    replay after new inputs are written gives that new batch's result."""
+    from token_dispatch_combine_b200 import MoERoundTrip
+    wl = W("graph", T=200, H=256, I=256, E=8, k=2, R=4, dtype=dtype, seed=20)
+    layer = DeviceLayer(wl)
+    dt = layer.x_dev.dtype
+    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt)
+    x = layer.x_dev.clone()
+    lg = layer.logits_dev.clone()
+    want1 = rt.forward(x, lg, layer.w_gate, layer.w_up, layer.w_down).clone()
+    g = rt.capture(x, lg, layer.w_gate, layer.w_up, layer.w_down)
+    rt.y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(rt.y, want1)
+    x2 = torch.randn_like(x.float()).to(dt)
+    lg2 = torch.randn_like(lg)
+    want2 = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt).forward(x2, lg2, layer.w_gate, layer.w_up,
+                                                                          layer.w_down).clone()
+    x.copy_(x2)
+    lg.copy_(lg2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(rt.y, want2)

@@ -190,7 +190,23 @@ class MoERoundTrip:
         self.down(w_down, stream)
         return self.combine(stream, y)
 
-    KERNELS_PER_FORWARD = 6  # route, dispatch x2, gate/up, down, combine
+    KERNELS_PER_FORWARD = 5  # route, dispatch, gate/up, down, combine
+
+    def capture(self, x, logits, w_gate, w_up, w_down, y=None, stream=None):
+        """Record ``forward`` on these fixed buffers into a CUDA graph.
+
+        Returns a ``torch.cuda.CUDAGraph``; ``graph.replay()`` reruns the whole
+        round trip on whatever ``x`` and ``logits`` then hold, with one launch
+        from the host.  Call ``forward`` once before capturing (the library sets
+        kernel attributes on first use, which must not happen during capture).
+        """
+        g = torch.cuda.CUDAGraph()
+        s = stream if stream is not None else torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.graph(g, stream=s):
+            self.forward(x, logits, w_gate, w_up, w_down, stream=s, y=y)
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        return g
 
 
 class MoEHostPipeline:

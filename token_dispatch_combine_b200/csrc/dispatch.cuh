@@ -9,17 +9,18 @@
 // [r*E/R, (r+1)*E/R), so the expert-major row order is rank-major.
 //
 // One cooperative launch (every CTA resident at once), three phases split by
-// two bounded grid barriers:
+// one or two bounded grid barriers:
 //  1. per chunk of <= 512 slots (chunks never straddle a source rank, token
 //     t's source rank being t*R/T): each slot's stable rank among the
 //     same-expert slots of its chunk, without atomics -- __match_any_sync
 //     groups a warp's lanes by expert, popc of the lower peers gives the
 //     in-warp rank, a per-expert scan over the CTA's warps adds the earlier
 //     warps' counts -- and the chunk's per-expert counts;
-//  2. one warp per expert scans that expert's counts over the chunks (warp
-//     prefix sums, 32 chunks per round) into per-chunk bases and a total;
-//     after the second barrier every CTA scans the E totals into expert
-//     offsets in shared memory;
+//  2. per-chunk bases (earlier chunks' counts of the same expert) and expert
+//     offsets: when the [chunks][E] count table is small (<= 8192 entries)
+//     every CTA loads it into shared memory and scans it itself; otherwise one
+//     warp per expert scans its column (warp prefix sums, 32 chunks a round)
+//     and, after a second barrier, every CTA scans the E totals;
 //  3. one warp per (token, slice of 128 16-byte columns) computes the token's
 //     k rows (offset + chunk base + in-chunk rank), writes the permutation
 //     (first slice only), and copies its slice of the token row to the k rows
@@ -38,6 +39,14 @@ constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kScatterVecsPerLane = 4;                   // 16-byte vectors in flight per lane
 constexpr int kScatterSlice = 32 * kScatterVecsPerLane;  // 16-byte vectors of a row per warp item
 constexpr uint64_t kGridBarrierLimitNs = 1000000000ull;   // 1 s
+// Count tables up to this many entries are scanned by every CTA in shared
+// memory, which saves the second grid barrier.
+constexpr size_t kSmallCountTable = 8192;
+
+__host__ __device__ __forceinline__ size_t dispatch_smem_table(int nchunks, int E) {
+  const size_t warps = (size_t)kDispatchWarps * E, table = (size_t)nchunks * E;
+  return (table <= kSmallCountTable && table > warps) ? table : warps;
+}
 
 struct DispatchGeom {
   int T, k, E, R, S;
@@ -151,7 +160,8 @@ __device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok) {
   return *s_ok != 0;
 }
 
-// Dynamic shared memory: warp_counts[kDispatchWarps][E] int32, then offs[E + 1].
+// Dynamic shared memory: warp_counts[kDispatchWarps][E] int32 (or the whole
+// [nchunks][E] table when it is small and larger), then offs[E + 1].
 template <typename T>
 __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
     DispatchGeom g, int H, int nslices, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
@@ -159,8 +169,10 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
     int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_to_row,
     int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
   extern __shared__ int32_t smem_i32[];
-  int32_t* warp_counts = smem_i32;                          // [kDispatchWarps][E]
-  int32_t* offs = smem_i32 + (size_t)kDispatchWarps * g.E;  // [E + 1]
+  int32_t* warp_counts = smem_i32;                                    // [kDispatchWarps][E]
+  int32_t* offs = smem_i32 + dispatch_smem_table(g.nchunks, g.E);     // [E + 1]
+  const bool small_table = (size_t)g.nchunks * g.E <= kSmallCountTable;
+  int32_t* cbase = smem_i32;  // small_table: [nchunks][E] chunk bases (reuses warp_counts)
   __shared__ int s_ok;
   pdl_wait();
   pdl_trigger();
@@ -221,6 +233,21 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
   }
   if (!grid_barrier(ws, &s_ok)) return;
 
+  if (small_table) {
+    // ---- phase 2 (small count table): every CTA scans the whole table itself
+    for (int i = threadIdx.x; i < g.nchunks * g.E; i += kDispatchThreads) cbase[i] = __ldcg(ws.chunk_counts + i);
+    __syncthreads();
+    for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) {
+      int run = 0;
+      for (int c = 0; c < g.nchunks; ++c) {
+        const int v = cbase[c * g.E + xx];
+        cbase[c * g.E + xx] = run;
+        run += v;
+      }
+      offs[xx] = run;
+      if (blockIdx.x == 0) expert_counts[xx] = run;
+    }
+  } else {
   // ---- phase 2a: one warp per expert, prefix over chunks
   for (size_t e = gwarp; e < (size_t)g.E; e += nwarps_grid) {
     int carry = 0;
@@ -245,6 +272,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
 
   // ---- phase 2b: expert offsets (every CTA, in shared memory)
   for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) offs[xx] = __ldcg(ws.totals + xx);
+  }
   __syncthreads();
   if (warp == 0) {
     int carry = 0;
@@ -273,12 +301,23 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
     if (threadIdx.x == 0) rank_offsets[g.R] = placed;
   }
   if (src_expert_counts) {  // a source rank's chunks are contiguous: differences of the chunk bases
-    for (size_t i = gtid; i < (size_t)g.R * g.E; i += nthreads_grid) {
-      const int r = (int)(i / g.E), xx = (int)(i - (size_t)r * g.E);
-      const int lo = __ldcg(ws.chunk_base + (size_t)(r * g.cpr) * g.E + xx);
-      const int hi = (r + 1 < g.R) ? __ldcg(ws.chunk_base + (size_t)((r + 1) * g.cpr) * g.E + xx)
-                                   : offs[xx + 1] - offs[xx];
-      src_expert_counts[i] = hi - lo;
+    if (small_table) {
+      if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < g.R * g.E; i += kDispatchThreads) {
+          const int r = i / g.E, xx = i - r * g.E;
+          const int lo = cbase[(r * g.cpr) * g.E + xx];
+          const int hi = (r + 1 < g.R) ? cbase[((r + 1) * g.cpr) * g.E + xx] : offs[xx + 1] - offs[xx];
+          src_expert_counts[i] = hi - lo;
+        }
+      }
+    } else {
+      for (size_t i = gtid; i < (size_t)g.R * g.E; i += nthreads_grid) {
+        const int r = (int)(i / g.E), xx = (int)(i - (size_t)r * g.E);
+        const int lo = __ldcg(ws.chunk_base + (size_t)(r * g.cpr) * g.E + xx);
+        const int hi = (r + 1 < g.R) ? __ldcg(ws.chunk_base + (size_t)((r + 1) * g.cpr) * g.E + xx)
+                                     : offs[xx + 1] - offs[xx];
+        src_expert_counts[i] = hi - lo;
+      }
     }
   }
   // rows past the last placed row (only when ids were dropped) get row_to_slot = -1
@@ -292,8 +331,10 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
       const int s = t * g.k + lane;
       const int e = __ldg(ids + s);
       const int rk = __ldcg(ws.slot_rank + s);
-      if (e >= 0 && e < g.E && rk >= 0)
-        my_row = offs[e] + __ldcg(ws.chunk_base + (size_t)chunk_of_slot(g, s) * g.E + e) + rk;
+      if (e >= 0 && e < g.E && rk >= 0) {
+        const size_t cb = (size_t)chunk_of_slot(g, s) * g.E + e;
+        my_row = offs[e] + (small_table ? cbase[cb] : __ldcg(ws.chunk_base + cb)) + rk;
+      }
       if (cs == 0) {
         slot_to_row[s] = my_row;
         if (my_row >= 0) row_to_slot[my_row] = s;
@@ -334,14 +375,14 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
                             int32_t* src_expert_counts, cudaStream_t stream) {
   DispatchWs ws = dispatch_ws_carve(workspace, g);
   auto kern = dispatch_kernel<T>;
-  const size_t smem = sizeof(int32_t) * ((size_t)kDispatchWarps * g.E + g.E + 1);
+  const size_t smem = sizeof(int32_t) * (dispatch_smem_table(g.nchunks, g.E) + g.E + 1);
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   static int attr_dev = -1;
   if (attr_dev != dev) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)(sizeof(int32_t) * ((size_t)kDispatchWarps * 1024 + 1025)));
+                               (int)(sizeof(int32_t) * (dispatch_smem_table(1, 1024) + 1025)));
     if (err != cudaSuccess) return err;
     attr_dev = dev;
   }
@@ -365,11 +406,13 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   cfg.blockDim = dim3(kDispatchThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = MOE_PDL ? 2 : 1;
   err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, x, ids, ws, x_disp, expert_counts, expert_offsets, rank_counts,
                            rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
   return err != cudaSuccess ? err : cudaGetLastError();
