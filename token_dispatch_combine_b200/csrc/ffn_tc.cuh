@@ -7,7 +7,8 @@
 // Improve Transformer"): h = SiLU(x Wg) * (x Wu), y = h Wd.
 //
 // Ragged expert segments: expert e owns rows [off[e], off[e+1]) of the
-// dispatched buffer, unpadded.  Every CTA rebuilds the tile list on the
+// dispatched buffer, unpadded.  An expert's last tile, when it holds at most
+// 64 rows, runs as an M=64 UMMA (half the tensor time of M=128).  Every CTA rebuilds the tile list on the
 // device from off[] (per-expert 128-row m-tiles, prefix-summed in shared
 // memory) so the host never reads the counts.  A 128-row tile may run past
 // its expert's last row: those extra rows are loaded (harmless: they belong to
@@ -53,6 +54,13 @@
 #endif
 #ifndef MOE_TC_HINT_B
 #define MOE_TC_HINT_B 0
+#endif
+//  MOE_TC_M64: tiles with at most 64 valid rows (an expert's last, partial
+//    tile) issue M=64 UMMAs, which take about half the time of M=128; the
+//    accumulator then sits in TMEM lanes 0-15 of each 32-lane quarter, so
+//    epilogue warp q holds rows 16q..16q+15 in its lanes 0-15.
+#ifndef MOE_TC_M64
+#define MOE_TC_M64 1
 #endif
 //  MOE_TC_DOWN_BN: force the down-projection n-tile width (0 = chosen from H).
 #ifndef MOE_TC_DOWN_BN
@@ -408,11 +416,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, C::MMA_N);
+      constexpr uint32_t idesc128 = idesc_bf16_f32(BM, C::MMA_N);
+      constexpr uint32_t idesc64 = idesc_bf16_f32(64, C::MMA_N);
       int stage = 0, local = 0;
       uint32_t phase = 0;
       bool ok = true, issued = false;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++local) {
+        uint32_t idesc = idesc128;
+        if (MOE_TC_M64) {
+          int e_, m0_, mend_, n0_;
+          tile_coords(tile, e_, m0_, mend_, n0_);
+          if (mend_ - m0_ <= 64) idesc = idesc64;
+        }
         const int acc = local & 1;
         const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, s_abort)) {
@@ -464,8 +479,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       int e, m0, mend, n0;
       tile_coords(tile, e, m0, mend, n0);
-      const int row = m0 + q * 32 + lane;
-      const bool row_ok = row < mend;
+      const bool m64 = MOE_TC_M64 && (mend - m0 <= 64);
+      const int row = m64 ? m0 + q * 16 + lane : m0 + q * 32 + lane;
+      const bool row_ok = row < mend && (!m64 || lane < 16);
       const uint32_t t_base = tmem_base + (uint32_t)acc * kAccStride + ((uint32_t)(q * 32) << 16);
       __nv_bfloat16* out_row = p.out + (size_t)row * p.N;
       constexpr int NCHUNK = (BN + 31) / 32;
