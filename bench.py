@@ -150,11 +150,13 @@ def barrier(world):
 
 
 def max_over_ranks(values, world):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's time)."""
     import torch
     if world == 1:
         return list(values)
     import torch.distributed as dist
-    t = torch.tensor(values, dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.tolist()
 
