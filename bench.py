@@ -47,7 +47,7 @@ def load_peaks():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for name in ("ffn_tc.cuh", "common.cuh"):
+    for name in ("ffn_tc.cuh", "ffn_tc2.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "token_dispatch_combine_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -239,7 +239,7 @@ def config_dict(wl):
 def run_ours(args, wl):
     import torch
 
-    from token_dispatch_combine_b200 import MoERoundTrip, moe_get_error
+    from token_dispatch_combine_b200 import FFN_TILING_PAIR, MoERoundTrip, moe_ffn_tiling_for, moe_get_error
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", torch.cuda.current_device())
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -385,6 +385,7 @@ def run_ours(args, wl):
     dc_gbs = (alg["dispatch_bytes"] + alg["combine_bytes"]) / ((t_disp + t_comb) * 1e-3) / 1e9
     gu_tflops = alg["gateup_flops"] / (t_gu * 1e-3) / 1e12
     peak_tf = peaks["bf16_tflops"]
+    tiling = moe_ffn_tiling_for(wl.E, wl.S)
     cpu = None
     if args.cpu_baseline and world == 1:
         rng = np.random.default_rng(1)
@@ -416,9 +417,12 @@ def run_ours(args, wl):
             "stage_timing": "per-stage CUDA events in a separate pass of the same steps (each stage boundary "
                             "adds event overhead); back_to_back: one event pair around dispatch+combine; stream: 20 dispatch+combine pairs over 4 buffer sets (>L2) under one event pair",
             "grouped_gemm_tflops": gemm_tflops, "grouped_gemm_frac_bf16": gemm_tflops / peak_tf,
+            "ffn_tiling": "pair" if tiling == FFN_TILING_PAIR else "single",
         },
         "roofline": {
-            "kernel": "grouped_gemm_tc_kernel<gate/up, SwiGLU epilogue>",
+            "kernel": ("grouped_gemm_tc2_kernel<gate/up, SwiGLU epilogue> (256-row tiles on 2-SM clusters)"
+                       if tiling == FFN_TILING_PAIR else
+                       "grouped_gemm_tc_kernel<gate/up, SwiGLU epilogue> (128-row tiles)"),
             "bound": "tensor", "achieved": gu_tflops, "peak": peak_tf, "unit": "TFLOP/s",
             "frac": gu_tflops / peak_tf, "traffic": dram_traffic(wl.name),
             "peak_source": f"{peak_src} bf16 dense (burst)",

@@ -178,6 +178,30 @@ moe_status moe_expert_ffn(const void* x_disp, int dtype, const void* w_gate, con
                           const void* w_down, const int32_t* expert_offsets, int E, int H, int I, int S, void* h,
                           void* y_disp, void* stream);
 
+/*
+ * Tile shape of the bf16 expert FFN (moe_expert_ffn, moe_ffn_gate_up,
+ * moe_ffn_down).  One setting for the whole process, read at each call.
+ *   MOE_FFN_TILING_AUTO    pair tiles when S >= 384 * E (enough rows per expert
+ *                          that padding each expert to 256 rows costs little),
+ *                          else single tiles.  The default.
+ *   MOE_FFN_TILING_SINGLE  128-row tiles, one SM per tile.
+ *   MOE_FFN_TILING_PAIR    256-row tiles computed by a cluster of two SMs
+ *                          (tcgen05 cta_group::2; each SM loads half of the
+ *                          weight tile); an expert's last tile with at most
+ *                          128 rows left uses an M = 128 pair MMA.
+ * Both shapes form the same products and accumulate them in float32 in the
+ * same K order.  float32 calls ignore the setting.
+ * moe_set_ffn_tiling returns MOE_ERR_INVALID_ARG for any other mode and keeps
+ * the old one.  moe_ffn_tiling_for returns the shape (SINGLE or PAIR) that a
+ * bf16 call with E experts and S rows would use now, or -1 for E <= 0 or S < 0.
+ */
+#define MOE_FFN_TILING_AUTO 0
+#define MOE_FFN_TILING_SINGLE 1
+#define MOE_FFN_TILING_PAIR 2
+moe_status moe_set_ffn_tiling(int mode);
+int moe_get_ffn_tiling(void);
+int moe_ffn_tiling_for(int E, int S);
+
 /* First half of moe_expert_ffn: h = SiLU(x_disp Wg_e) * (x_disp Wu_e). */
 moe_status moe_ffn_gate_up(const void* x_disp, int dtype, const void* w_gate, const void* w_up,
                            const int32_t* expert_offsets, int E, int H, int I, int S, void* h, void* stream);

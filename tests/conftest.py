@@ -25,3 +25,15 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+FFN_TILINGS = {"auto": 0, "single": 1, "pair": 2}  # moe_set_ffn_tiling modes
+
+
+@pytest.fixture
+def ffn_tiling(request):
+    """Force the bf16 FFN tile shape for one test (indirect parameter), back to auto afterwards."""
+    from token_dispatch_combine_b200 import moe_set_ffn_tiling
+    moe_set_ffn_tiling(FFN_TILINGS[request.param])
+    yield request.param
+    moe_set_ffn_tiling(0)

@@ -96,3 +96,29 @@ def test_ffn_and_combine_reject():
 def test_python_wrapper_raises_moe_error():
     with pytest.raises(_native.MoeError):
         _native.check(_native.lib().moe_route(FAKE, 4, 4, 9, FAKE, FAKE, None), "moe_route")
+
+
+def test_ffn_tiling_setting_is_host_only():
+    """The tiling mode is host state: set, read back, resolved by rows per expert."""
+    import token_dispatch_combine_b200 as moe
+    lib = _native.lib()
+    assert moe.moe_get_ffn_tiling() == moe.FFN_TILING_AUTO
+    try:
+        # auto: pair tiles from 384 rows per expert on
+        assert moe.moe_ffn_tiling_for(32, 16384) == moe.FFN_TILING_PAIR
+        assert moe.moe_ffn_tiling_for(32, 384 * 32) == moe.FFN_TILING_PAIR
+        assert moe.moe_ffn_tiling_for(32, 384 * 32 - 1) == moe.FFN_TILING_SINGLE
+        assert moe.moe_ffn_tiling_for(256, 65536) == moe.FFN_TILING_SINGLE
+        assert moe.moe_ffn_tiling_for(0, 10) == -1
+        for mode in (moe.FFN_TILING_SINGLE, moe.FFN_TILING_PAIR):
+            moe.moe_set_ffn_tiling(mode)
+            assert moe.moe_get_ffn_tiling() == mode
+            assert moe.moe_ffn_tiling_for(256, 1) == mode
+            assert moe.moe_ffn_tiling_for(1, 1 << 20) == mode
+        assert lib.moe_set_ffn_tiling(3) == _native.MOE_ERR_INVALID_ARG
+        assert lib.moe_set_ffn_tiling(-1) == _native.MOE_ERR_INVALID_ARG
+        assert moe.moe_get_ffn_tiling() == moe.FFN_TILING_PAIR  # unchanged by the rejected calls
+        with pytest.raises(moe.MoeError):
+            moe.moe_set_ffn_tiling(7)
+    finally:
+        moe.moe_set_ffn_tiling(moe.FFN_TILING_AUTO)

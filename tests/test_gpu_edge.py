@@ -116,8 +116,9 @@ def test_combine_skips_out_of_range_rows():
     np.testing.assert_allclose(yn[3], 0.5 * ydn[6] + 0.5 * ydn[7], rtol=1e-6)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_ffn_clamps_inconsistent_offsets(dtype):
+@pytest.mark.parametrize("dtype,ffn_tiling", [(torch.float32, "auto"), (torch.bfloat16, "single"),
+                                              (torch.bfloat16, "pair")], indirect=["ffn_tiling"])
+def test_ffn_clamps_inconsistent_offsets(dtype, ffn_tiling):
     m = _api()
     E, H, I, S = 4, 64, 64, 40
     x = torch.randn(S, H, device="cuda").to(dtype)

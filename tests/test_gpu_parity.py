@@ -60,8 +60,9 @@ def check_routing_and_dispatch(layer: DeviceLayer, rt):
     return ids, w, ref, x_disp
 
 
+@pytest.mark.parametrize("ffn_tiling", ["single", "pair"], indirect=True)
 @pytest.mark.parametrize("name", sorted(SMALL))
-def test_small_layer_full_parity(name):
+def test_small_layer_full_parity(name, ffn_tiling):
     wl = SMALL[name]
     layer = DeviceLayer(wl)
     rt = run_gpu(layer)
@@ -89,6 +90,17 @@ def _sample_rows(offsets, counts, S, rng, n_random=24):
 
 @pytest.mark.parametrize("name", ["gptoss_uniform", "gptoss_zipf", "dsr1_decode", "dsr1_prefill"])
 def test_full_size_layer(name):
+    check_full_size_layer(name)
+
+
+@pytest.mark.parametrize("ffn_tiling,name", [("single", "gptoss_zipf"), ("pair", "dsr1_decode"),
+                                              ("pair", "dsr1_prefill")], indirect=["ffn_tiling"])
+def test_full_size_layer_other_tiling(name, ffn_tiling):
+    """The full-size layers again with the tile shape that auto does not pick for them."""
+    check_full_size_layer(name)
+
+
+def check_full_size_layer(name):
     wl = synth.WORKLOADS[name]
     layer = DeviceLayer(wl)
     rt = run_gpu(layer)
@@ -117,6 +129,26 @@ def test_full_size_layer(name):
     assert torch.isfinite(rt.y.float()).all()
 
 
+def test_single_and_pair_tiles_agree_bit_for_bit():
+    """Both tile shapes form the same products in the same K order: h and y_disp
+    are identical, including at expert boundaries, half tiles and N tails."""
+    from token_dispatch_combine_b200 import MoERoundTrip, moe_set_ffn_tiling
+    for wl in (SMALL["bf16_multi_tile"], SMALL["bf16_ragged_n"], synth.WORKLOADS["gptoss_zipf"]):
+        layer = DeviceLayer(wl)
+        outs = []
+        try:
+            for mode in (1, 2):
+                moe_set_ffn_tiling(mode)
+                rt = run_gpu(layer, MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, layer.x_dev.dtype))
+                outs.append([t.view(torch.int16).clone() for t in (rt.h, rt.y_disp, rt.y)])
+        finally:
+            moe_set_ffn_tiling(0)
+        for a, b in zip(*outs):
+            assert torch.equal(a, b), wl.name
+        del layer, outs
+        torch.cuda.empty_cache()
+
+
 def test_repeated_calls_are_identical():
     wl = SMALL["bf16_multi_tile"]
     layer = DeviceLayer(wl)
@@ -127,7 +159,8 @@ def test_repeated_calls_are_identical():
         assert (a == dev_to_np(t)).all()
 
 
-def test_all_tokens_to_one_expert():
+@pytest.mark.parametrize("ffn_tiling", ["single", "pair"], indirect=True)
+def test_all_tokens_to_one_expert(ffn_tiling):
     wl = W("one_hot", T=300, H=128, I=128, E=8, k=1, R=2, dtype="bf16", seed=17)
     logits = np.zeros((wl.T, wl.E), np.float32)
     logits[:, 5] = 1.0
@@ -178,8 +211,9 @@ def test_host_pipeline_matches_forward():
         assert torch.equal(yh, y.view(torch.int16).cpu())
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_graph_replay_matches_forward(dtype):
+@pytest.mark.parametrize("dtype,ffn_tiling", [("bf16", "single"), ("bf16", "pair"), ("f32", "auto")],
+                         indirect=["ffn_tiling"])
+def test_graph_replay_matches_forward(dtype, ffn_tiling):
     """The whole round trip captured in a CUDA graph gives the eager result, and a
     replay after new inputs are written gives that new batch's result."""
     from token_dispatch_combine_b200 import MoERoundTrip

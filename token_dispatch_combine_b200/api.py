@@ -140,6 +140,22 @@ def moe_combine(y_disp, topk_w, slot_to_row, y, stream=None):
     return y
 
 
+def moe_set_ffn_tiling(mode: int) -> None:
+    """Tile shape of the bf16 expert FFN for the whole process:
+    FFN_TILING_AUTO (0), FFN_TILING_SINGLE (1, 128-row tiles on one SM) or
+    FFN_TILING_PAIR (2, 256-row tiles on a 2-SM cluster)."""
+    check(_native.lib().moe_set_ffn_tiling(int(mode)), "moe_set_ffn_tiling")
+
+
+def moe_get_ffn_tiling() -> int:
+    return _native.lib().moe_get_ffn_tiling()
+
+
+def moe_ffn_tiling_for(E: int, S: int) -> int:
+    """The tile shape (SINGLE or PAIR) a bf16 FFN call with E experts and S rows would use now."""
+    return _native.lib().moe_ffn_tiling_for(int(E), int(S))
+
+
 def moe_get_error(stream=None) -> tuple[int, int]:
     """Synchronise the stream; return (status, error-word bits) and clear the word."""
     bits = ctypes.c_uint32(0)

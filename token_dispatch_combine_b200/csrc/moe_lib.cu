@@ -3,6 +3,7 @@
 // Host side only validates arguments, picks kernel configurations and
 // enqueues launches on the caller's stream.  It never allocates, never copies
 // to the host and never synchronises (moe_get_error excepted).
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 #include <string>
@@ -12,9 +13,23 @@
 #include "dispatch.cuh"
 #include "ffn_simt.cuh"
 #include "ffn_tc.cuh"
+#include "ffn_tc2.cuh"
 #include "route.cuh"
 
 namespace {
+
+std::atomic<int> g_ffn_tiling{MOE_FFN_TILING_AUTO};
+
+// Pair tiles pad each expert's rows to 256 instead of 128; they pay off once
+// the average expert holds enough rows (measured: 512 rows per expert gain,
+// 256 lose).
+constexpr int kPairMinRowsPerExpert = 384;
+
+int resolve_tiling(int E, int S) {
+  const int mode = g_ffn_tiling.load(std::memory_order_relaxed);
+  if (mode != MOE_FFN_TILING_AUTO) return mode;
+  return (long long)S >= (long long)kPairMinRowsPerExpert * E ? MOE_FFN_TILING_PAIR : MOE_FFN_TILING_SINGLE;
+}
 
 thread_local std::string g_last_msg;
 
@@ -54,6 +69,17 @@ moe_status check_k_e(int k, int E) {
 extern "C" {
 
 int moe_abi_version(void) { return 1; }
+
+moe_status moe_set_ffn_tiling(int mode) {
+  if (mode != MOE_FFN_TILING_AUTO && mode != MOE_FFN_TILING_SINGLE && mode != MOE_FFN_TILING_PAIR)
+    return fail(MOE_ERR_INVALID_ARG, "moe_set_ffn_tiling: mode must be 0 (auto), 1 (single) or 2 (pair)");
+  g_ffn_tiling.store(mode, std::memory_order_relaxed);
+  return MOE_OK;
+}
+
+int moe_get_ffn_tiling(void) { return g_ffn_tiling.load(std::memory_order_relaxed); }
+
+int moe_ffn_tiling_for(int E, int S) { return E > 0 && S >= 0 ? resolve_tiling(E, S) : -1; }
 
 const char* moe_status_string(int status) {
   switch (status) {
@@ -216,7 +242,9 @@ moe_status moe_ffn_gate_up(const void* x_disp, int dtype, const void* w_gate, co
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t err;
   if (dtype == MOE_BF16)
-    err = moe::tc::launch_gate_up(x_disp, w_gate, w_up, expert_offsets, E, H, I, S, h, s);
+    err = resolve_tiling(E, S) == MOE_FFN_TILING_PAIR
+              ? moe::tc::launch_gate_up_pair(x_disp, w_gate, w_up, expert_offsets, E, H, I, S, h, s)
+              : moe::tc::launch_gate_up(x_disp, w_gate, w_up, expert_offsets, E, H, I, S, h, s);
   else
     err = moe::launch_ffn_simt_gate_up((const float*)x_disp, (const float*)w_gate, (const float*)w_up,
                                        expert_offsets, E, H, I, S, (float*)h, s);
@@ -233,7 +261,9 @@ moe_status moe_ffn_down(const void* h, int dtype, const void* w_down, const int3
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t err;
   if (dtype == MOE_BF16)
-    err = moe::tc::launch_down(h, w_down, expert_offsets, E, H, I, S, y_disp, s);
+    err = resolve_tiling(E, S) == MOE_FFN_TILING_PAIR
+              ? moe::tc::launch_down_pair(h, w_down, expert_offsets, E, H, I, S, y_disp, s)
+              : moe::tc::launch_down(h, w_down, expert_offsets, E, H, I, S, y_disp, s);
   else
     err = moe::launch_ffn_simt_down((const float*)h, (const float*)w_down, expert_offsets, E, H, I, S,
                                     (float*)y_disp, s);
