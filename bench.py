@@ -239,7 +239,9 @@ def config_dict(wl):
 def run_ours(args, wl):
     import torch
 
-    from token_dispatch_combine_b200 import FFN_TILING_PAIR, MoERoundTrip, moe_ffn_tiling_for, moe_get_error
+    from token_dispatch_combine_b200 import (FFN_TILING_PAIR, MoERoundTrip, moe_ffn_tiling_for, moe_get_error,
+                                             moe_set_ffn_tiling)
+    moe_set_ffn_tiling({"auto": 0, "single": 1, "pair": 2}[args.ffn_tiling])
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", torch.cuda.current_device())
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -446,6 +448,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="gptoss_uniform", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ffn-tiling", default="auto", choices=["auto", "single", "pair"],
+                    help="tile shape of the bf16 expert FFN (moe_set_ffn_tiling); auto picks by rows per expert")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false",
                     help="skip the CPU oracle leg (used for profiler runs)")
     args = ap.parse_args()
