@@ -232,7 +232,7 @@ def run_reference(args, wl):
 def config_dict(wl):
     return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k, "R": wl.R,
             "dtype": wl.dtype, "routing_bias": wl.bias, "seed": wl.seed,
-            "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)"}
+            "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, then read back)"}
 
 
 # --------------------------------------------------------------------------- our arm
@@ -256,6 +256,7 @@ def run_ours(args, wl):
     wg, wu, wd = up(wg_np), up(wu_np), up(wd_np)
     rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(ev):
@@ -272,10 +273,14 @@ def run_ours(args, wl):
         ev[5].record(stream)
 
     def flush_and_hold():
-        # Outside the timed events: evict L2, then keep the GPU busy for ~0.2 ms so
-        # the host has enqueued the whole step before the GPU reaches it (the stage
-        # events then measure GPU time, not Python call overhead).
+        # Outside the timed events: evict L2 by writing a buffer 4x its size, then
+        # read that buffer back so L2 holds clean lines of it (a write alone leaves
+        # ~126 MB of dirty lines that the timed step would have to write back);
+        # then keep the GPU busy for ~0.2 ms so the host has enqueued the whole
+        # step before the GPU reaches it (the stage events then measure GPU time,
+        # not Python call overhead).
         flush.zero_()
+        torch.sum(flush, dim=0, out=flush_sum)
         torch.cuda._sleep(HOLD_CYCLES)
 
     for _ in range(args.warmup):
