@@ -122,3 +122,18 @@ def test_ffn_tiling_setting_is_host_only():
             moe.moe_set_ffn_tiling(7)
     finally:
         moe.moe_set_ffn_tiling(moe.FFN_TILING_AUTO)
+
+
+def test_library_override_variable_is_honoured(tmp_path):
+    """MOE_B200_LIBRARY names a prebuilt copy of the library to load instead of the in-tree build."""
+    import shutil
+    import subprocess
+    import sys
+    copy = tmp_path / "libmoe_copy.so"
+    shutil.copy(_native._build.build(), copy)
+    code = ("import token_dispatch_combine_b200 as m; "
+            "print(m._native.library_path()); print(m._native.lib().moe_abi_version())")
+    env = dict(os.environ, MOE_B200_LIBRARY=str(copy))
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, check=True,
+                         cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__)))).stdout.split()
+    assert out[0] == str(copy) and int(out[1]) >= 1

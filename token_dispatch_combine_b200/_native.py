@@ -7,6 +7,7 @@ importing the package raises.
 from __future__ import annotations
 
 import ctypes
+import os
 import threading
 
 from . import build as _build
@@ -62,11 +63,13 @@ def _configure(lib):
 
 
 def lib():
-    """The loaded library (built in-tree first if missing or stale)."""
+    """The loaded library: the file named by MOE_B200_LIBRARY if that is set
+    (a prebuilt copy of this library), else the in-tree build (built first if
+    missing or stale)."""
     global _lib
     with _lock:
         if _lib is None:
-            path = _build.build()
+            path = os.environ.get("MOE_B200_LIBRARY") or _build.build()
             _lib = _configure(ctypes.CDLL(path))
     return _lib
 
@@ -78,4 +81,4 @@ def check(status: int, fn: str):
 
 
 def library_path() -> str:
-    return _build.LIB_PATH
+    return os.environ.get("MOE_B200_LIBRARY") or _build.LIB_PATH

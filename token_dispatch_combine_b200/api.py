@@ -168,7 +168,8 @@ class MoERoundTrip:
 
     Route -> dispatch -> grouped SwiGLU FFN -> combine, all on `stream`.
     Device memory for every intermediate is allocated once here (through
-    torch); ``forward`` enqueues six kernels and allocates nothing.
+    torch); ``forward`` enqueues five kernels (route, dispatch, gate/up, down,
+    combine) and allocates nothing.
     """
 
     def __init__(self, T, H, I, E, k, R, dtype, device="cuda", src_counts=True):

@@ -21,11 +21,13 @@
 //     every CTA loads it into shared memory and scans it itself; otherwise one
 //     warp per expert scans its column (warp prefix sums, 32 chunks a round)
 //     and, after a second barrier, every CTA scans the E totals;
-//  3. one warp per (token, slice of 128 16-byte columns) computes the token's
-//     k rows (offset + chunk base + in-chunk rank), writes the permutation
-//     (first slice only), and copies its slice of the token row to the k rows
-//     with 16-byte vector accesses.  Each warp loads its first slice of x
-//     before phase 1, so that read overlaps the counting and the barriers.
+//  3. each CTA owns a contiguous range of tokens: one thread per slot computes
+//     the slot's row (offset + chunk base + in-chunk rank) into shared memory
+//     and writes the permutation, then one warp per (token, slice of 128
+//     16-byte columns) copies its slice of the token row to the k rows with
+//     16-byte vector accesses.  Before phase 1 each CTA asks L2 for its token
+//     rows of x and each warp loads its first slice, so those reads overlap
+//     the counting and the barriers.
 // A barrier that does not complete within 1 s sets the timeout bit of the
 // device error word; the kernel then returns without writing the rows.
 #pragma once
@@ -38,6 +40,7 @@ constexpr int kDispatchThreads = 512;
 constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kScatterVecsPerLane = 4;                   // 16-byte vectors in flight per lane
 constexpr int kScatterSlice = 32 * kScatterVecsPerLane;  // 16-byte vectors of a row per warp item
+constexpr int kRowRound = kDispatchThreads / 8;          // tokens per phase-3 round: one slot per thread at k <= 8
 constexpr uint64_t kGridBarrierLimitNs = 1000000000ull;   // 1 s
 // Count tables up to this many entries are scanned by every CTA in shared
 // memory, which saves the second grid barrier.
@@ -161,19 +164,34 @@ __device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok) {
 }
 
 // Dynamic shared memory: warp_counts[kDispatchWarps][E] int32 (or the whole
-// [nchunks][E] table when it is small and larger), then offs[E + 1].
+// [nchunks][E] table when it is small and larger), then offs[E + 1], then the
+// rows of one round of this CTA's slots, rows[kDispatchThreads].
 template <typename T>
 __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
-    DispatchGeom g, int H, int nslices, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
+    DispatchGeom g, int H, int nslices, int tpc, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
     T* __restrict__ x_disp, int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
     int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_to_row,
     int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
   extern __shared__ int32_t smem_i32[];
   int32_t* warp_counts = smem_i32;                                    // [kDispatchWarps][E]
   int32_t* offs = smem_i32 + dispatch_smem_table(g.nchunks, g.E);     // [E + 1]
+  int32_t* s_rows = offs + g.E + 1;                                    // [kDispatchThreads]
   const bool small_table = (size_t)g.nchunks * g.E <= kSmallCountTable;
   int32_t* cbase = smem_i32;  // small_table: [nchunks][E] chunk bases (reuses warp_counts)
   __shared__ int s_ok;
+  // ---- this CTA's tokens [tb, te): ask L2 for their rows of x.  A prefetch
+  // changes no data, so it may run before the previous kernel has finished.
+  constexpr int N = Vec16<T>::N;
+  const int nvec = H / N;
+  const int tb = min(g.T, (int)blockIdx.x * tpc), te = min(g.T, tb + tpc);
+  if (threadIdx.x == 0 && te > tb) {
+    const char* base = reinterpret_cast<const char*>(x + (size_t)tb * H);
+    const size_t bytes = (size_t)(te - tb) * H * sizeof(T);  // a multiple of 16 (H * sizeof(T) is)
+    for (size_t b = 0; b < bytes; b += 65536) {
+      const uint32_t n = (uint32_t)min((size_t)65536, bytes - b);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + b), "r"(n) : "memory");
+    }
+  }
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = (int)lane_id();
@@ -183,17 +201,14 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
   const size_t nthreads_grid = (size_t)gridDim.x * kDispatchThreads;
   if (threadIdx.x == 0) s_ok = 1;
 
-  // ---- prefetch this warp's first slice of x (it does not depend on the counts)
-  constexpr int N = Vec16<T>::N;
-  const int nvec = H / N;
-  const size_t nitems = (size_t)g.T * nslices;
+  // ---- each warp's first slice of x into registers (it does not depend on the counts)
   uint4 pre[kScatterVecsPerLane];
-  if (gwarp < nitems) {
-    const int t = (int)(gwarp / nslices), cs = (int)(gwarp - (size_t)t * nslices);
-    const char* src = reinterpret_cast<const char*>(x + (size_t)t * H);
+  const int pre_tok = tb + warp / nslices, pre_cs = warp % nslices;
+  if (pre_tok < min(te, tb + kRowRound)) {
+    const char* src = reinterpret_cast<const char*>(x + (size_t)pre_tok * H);
 #pragma unroll
     for (int u = 0; u < kScatterVecsPerLane; ++u) {
-      const int i = cs * kScatterSlice + u * 32 + lane;
+      const int i = pre_cs * kScatterSlice + u * 32 + lane;
       if (i < nvec) pre[u] = ld_nc_v4(src + (size_t)i * 16);
     }
   }
@@ -237,7 +252,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
     // ---- phase 2 (small count table): every CTA scans the whole table itself
     for (int i = threadIdx.x; i < g.nchunks * g.E; i += kDispatchThreads) cbase[i] = __ldcg(ws.chunk_counts + i);
     __syncthreads();
-    for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) {
+    for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) {  // thread per expert, prefix over chunks
       int run = 0;
       for (int c = 0; c < g.nchunks; ++c) {
         const int v = cbase[c * g.E + xx];
@@ -323,48 +338,52 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
   // rows past the last placed row (only when ids were dropped) get row_to_slot = -1
   for (size_t i = gtid; i < (size_t)(g.S - placed); i += nthreads_grid) row_to_slot[placed + i] = -1;
 
-  // ---- phase 3: rows
-  for (size_t item = gwarp; item < nitems; item += nwarps_grid) {
-    const int t = (int)(item / nslices), cs = (int)(item - (size_t)t * nslices);
-    int my_row = -1;
-    if (lane < g.k) {
-      const int s = t * g.k + lane;
+  // ---- phase 3: this CTA's tokens, kRowRound at a time
+  for (int r0 = tb; r0 < te; r0 += kRowRound) {
+    const int r1 = min(r0 + kRowRound, te);
+    const int nslot = (r1 - r0) * g.k;
+    if ((int)threadIdx.x < nslot) {
+      const int s = r0 * g.k + (int)threadIdx.x;
       const int e = __ldg(ids + s);
       const int rk = __ldcg(ws.slot_rank + s);
+      int row = -1;
       if (e >= 0 && e < g.E && rk >= 0) {
-        const size_t cb = (size_t)chunk_of_slot(g, s) * g.E + e;
-        my_row = offs[e] + (small_table ? cbase[cb] : __ldcg(ws.chunk_base + cb)) + rk;
+        const int c = chunk_of_slot(g, s);
+        const size_t cb = (size_t)c * g.E + e;
+        row = offs[e] + (small_table ? cbase[cb] : __ldcg(ws.chunk_base + cb)) + rk;
       }
-      if (cs == 0) {
-        slot_to_row[s] = my_row;
-        if (my_row >= 0) row_to_slot[my_row] = s;
+      s_rows[threadIdx.x] = row;
+      slot_to_row[s] = row;
+      if (row >= 0) row_to_slot[row] = s;
+    }
+    __syncthreads();
+    const int nit = (r1 - r0) * nslices;
+    for (int item = warp; item < nit; item += kDispatchWarps) {
+      const int tl = item / nslices, cs = item - tl * nslices;
+      uint4 v[kScatterVecsPerLane];
+      if (r0 == tb && item == warp) {  // the slice loaded before phase 1
+#pragma unroll
+        for (int u = 0; u < kScatterVecsPerLane; ++u) v[u] = pre[u];
+      } else {
+        const char* src = reinterpret_cast<const char*>(x + (size_t)(r0 + tl) * H);
+#pragma unroll
+        for (int u = 0; u < kScatterVecsPerLane; ++u) {
+          const int i = cs * kScatterSlice + u * 32 + lane;
+          if (i < nvec) v[u] = ld_nc_v4(src + (size_t)i * 16);
+        }
+      }
+      for (int j = 0; j < g.k; ++j) {
+        const int row = s_rows[tl * g.k + j];
+        if (row < 0) continue;
+        char* dst = reinterpret_cast<char*>(x_disp + (size_t)row * H);
+#pragma unroll
+        for (int u = 0; u < kScatterVecsPerLane; ++u) {
+          const int i = cs * kScatterSlice + u * 32 + lane;
+          if (i < nvec) st_v4(dst + (size_t)i * 16, v[u]);
+        }
       }
     }
-    int rows[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xFFFFFFFFu, my_row, j);
-    uint4 v[kScatterVecsPerLane];
-    if (item == gwarp) {
-#pragma unroll
-      for (int u = 0; u < kScatterVecsPerLane; ++u) v[u] = pre[u];
-    } else {
-      const char* src = reinterpret_cast<const char*>(x + (size_t)t * H);
-#pragma unroll
-      for (int u = 0; u < kScatterVecsPerLane; ++u) {
-        const int i = cs * kScatterSlice + u * 32 + lane;
-        if (i < nvec) v[u] = ld_nc_v4(src + (size_t)i * 16);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j >= g.k || rows[j] < 0) continue;
-      char* dst = reinterpret_cast<char*>(x_disp + (size_t)rows[j] * H);
-#pragma unroll
-      for (int u = 0; u < kScatterVecsPerLane; ++u) {
-        const int i = cs * kScatterSlice + u * 32 + lane;
-        if (i < nvec) st_v4(dst + (size_t)i * 16, v[u]);
-      }
-    }
+    __syncthreads();  // s_rows is reused by the next round
   }
 }
 
@@ -375,14 +394,14 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
                             int32_t* src_expert_counts, cudaStream_t stream) {
   DispatchWs ws = dispatch_ws_carve(workspace, g);
   auto kern = dispatch_kernel<T>;
-  const size_t smem = sizeof(int32_t) * (dispatch_smem_table(g.nchunks, g.E) + g.E + 1);
+  const size_t smem = sizeof(int32_t) * (dispatch_smem_table(g.nchunks, g.E) + g.E + 1 + kDispatchThreads);
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   static int attr_dev = -1;
   if (attr_dev != dev) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)(sizeof(int32_t) * (dispatch_smem_table(1, 1024) + 1025)));
+                               (int)(sizeof(int32_t) * (dispatch_smem_table(1, 1024) + 1025 + kDispatchThreads)));
     if (err != cudaSuccess) return err;
     attr_dev = dev;
   }
@@ -396,10 +415,14 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   if (cap < 1) return cudaErrorCooperativeLaunchTooLarge;
   const int nvec = H / Vec16<T>::N;
   const int nslices = (nvec + kScatterSlice - 1) / kScatterSlice;
-  const long long item_ctas = ((long long)g.T * nslices + kDispatchWarps - 1) / kDispatchWarps;
+  // phase 3: a CTA takes a contiguous token range; as many CTAs as keep every
+  // warp at one (token, slice) item, within the co-residency bound
+  const int tpc_one = kDispatchWarps / nslices > 0 ? kDispatchWarps / nslices : 1;
+  const long long item_ctas = ((long long)g.T + tpc_one - 1) / tpc_one;
   long long want = item_ctas > g.nchunks ? item_ctas : (long long)g.nchunks;
   if (want < 1) want = 1;
   const int grid = (int)(want < cap ? want : cap);
+  const int tpc = (g.T + grid - 1) / grid;  // tokens per CTA in phase 3
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -413,7 +436,7 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = MOE_PDL ? 2 : 1;
-  err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, x, ids, ws, x_disp, expert_counts, expert_offsets, rank_counts,
+  err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, tpc, x, ids, ws, x_disp, expert_counts, expert_offsets, rank_counts,
                            rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
