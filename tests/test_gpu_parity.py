@@ -31,6 +31,9 @@ SMALL = {
     "bf16_one_token": W("bf16_one_token", T=1, H=64, I=64, E=4, k=1, R=2, dtype="bf16", seed=14),
     "f32_top4": W("f32_top4", T=100, H=96, I=160, E=8, k=4, R=2, dtype="f32", seed=15),
     "bf16_top8_e256": W("bf16_top8_e256", T=96, H=128, I=128, E=256, k=8, R=32, dtype="bf16", seed=16),
+    # the largest expert count the calls accept, top-8: large dispatch count table
+    # (second grid barrier), 1024-expert tile prefix in the GEMMs' shared memory
+    "bf16_e1024": W("bf16_e1024", T=2048, H=128, I=192, E=1024, k=8, R=8, dtype="bf16", seed=21),
 }
 
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <utility>
 
 #include "moe_b200.h"
@@ -54,6 +56,51 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = MOE_PDL ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// ---- host-side per-device setup, safe to call from several host threads
+constexpr int kMaxDevices = 64;
+
+// Runs a setup step (e.g. raising a kernel's shared-memory limit) once per
+// device; a failed step is retried by the next call.
+class PerDeviceOnce {
+ public:
+  template <typename F>
+  cudaError_t run(int dev, F&& setup) {
+    if (dev < 0 || dev >= kMaxDevices) return setup();
+    if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    const cudaError_t err = setup();
+    if (err == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+    return err;
+  }
+
+ private:
+  std::mutex mu_;
+  std::atomic<bool> done_[kMaxDevices] = {};
+};
+
+// A positive per-device value computed once (e.g. an occupancy bound).
+class PerDeviceInt {
+ public:
+  template <typename F>
+  int get(int dev, F&& compute) {
+    if (dev < 0 || dev >= kMaxDevices) return compute();
+    int v = val_[dev].load(std::memory_order_acquire);
+    if (v > 0) return v;
+    v = compute();
+    if (v > 0) val_[dev].store(v, std::memory_order_release);
+    return v;
+  }
+
+ private:
+  std::atomic<int> val_[kMaxDevices] = {};
+};
+
+inline int current_device() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess ? dev : 0;
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

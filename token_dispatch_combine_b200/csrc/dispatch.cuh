@@ -395,16 +395,13 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   DispatchWs ws = dispatch_ws_carve(workspace, g);
   auto kern = dispatch_kernel<T>;
   const size_t smem = sizeof(int32_t) * (dispatch_smem_table(g.nchunks, g.E) + g.E + 1 + kDispatchThreads);
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  const int dev = current_device();
+  static PerDeviceOnce attr_once;  // raise the shared-memory limit once per device, for the largest E
+  cudaError_t err = attr_once.run(dev, [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(sizeof(int32_t) * (dispatch_smem_table(1, 1024) + 1025 + kDispatchThreads)));
+  });
   if (err != cudaSuccess) return err;
-  static int attr_dev = -1;
-  if (attr_dev != dev) {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)(sizeof(int32_t) * (dispatch_smem_table(1, 1024) + 1025 + kDispatchThreads)));
-    if (err != cudaSuccess) return err;
-    attr_dev = dev;
-  }
   // Co-residency bound of the cooperative grid for this shared-memory size.
   int per_sm = 0, sms = 0;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDispatchThreads, smem);

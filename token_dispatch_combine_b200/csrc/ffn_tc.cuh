@@ -553,15 +553,16 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (thread-safe static init).
 inline EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static const EncodeTiledFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    return (EncodeTiledFn) nullptr;
+  }();
   return fn;
 }
 
@@ -591,15 +592,14 @@ inline bool make_tmap_weight(CUtensorMap* m, const void* base, int E, int K, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SMs of the current device.
 inline int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
+  static PerDeviceInt sms;
+  const int dev = current_device();
+  return sms.get(dev, [&] {
+    int n = 0;
+    return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+  });
 }
 
 template <bool GATEUP, int BN, int STAGES>
@@ -608,19 +608,15 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUten
   using C = Cfg<GATEUP, BN, STAGES>;
   auto kern = grouped_gemm_tc_kernel<GATEUP, BN, STAGES>;
   const size_t smem = C::smem_bytes(p.E);
-  static int configured_dev = -1;  // the attribute is per device; set it once for the largest E
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_dev != dev) {
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)C::smem_bytes(1024));
-    if (err != cudaSuccess) return err;
-    configured_dev = dev;
-  }
+  static PerDeviceOnce attr_once;  // the attribute is per device; set it once for the largest E
+  cudaError_t err = attr_once.run(current_device(), [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem_bytes(1024));
+  });
+  if (err != cudaSuccess) return err;
   const long long max_tiles = ((long long)(p.S + BM - 1) / BM + p.E) * p.ntn;
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
-  cudaError_t err = launch_pdl(kern, grid, kThreads, smem, stream, ta, tb0, tb1, p);
+  err = launch_pdl(kern, grid, kThreads, smem, stream, ta, tb0, tb1, p);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

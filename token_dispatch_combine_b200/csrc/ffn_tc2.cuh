@@ -440,27 +440,24 @@ inline bool make_tmap_act64(CUtensorMap* m, const void* base, int rows, int K) {
 // SM), cached per device.
 template <bool GATEUP>
 int max_pair_clusters(size_t smem) {
-  static int cached_dev = -1, cached = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (cached_dev == dev) return cached;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * (num_sms() / 2));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tc2_kernel<GATEUP>, &cfg) != cudaSuccess || n <= 0)
-    n = num_sms() / 2;
-  cached = n;
-  cached_dev = dev;
-  return n;
+  static PerDeviceInt cached;
+  return cached.get(current_device(), [&] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tc2_kernel<GATEUP>, &cfg) != cudaSuccess || n <= 0)
+      n = num_sms() / 2;
+    return n;
+  });
 }
 
 template <bool GATEUP>
@@ -469,15 +466,11 @@ cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& ta64, const CUt
   using C = Cfg2<GATEUP>;
   auto kern = grouped_gemm_tc2_kernel<GATEUP>;
   const size_t smem = C::smem_bytes(p.E);
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_dev != dev) {
-    cudaError_t err =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem_bytes(1024));
-    if (err != cudaSuccess) return err;
-    configured_dev = dev;
-  }
+  static PerDeviceOnce attr_once;  // the attribute is per device; set it once for the largest E
+  cudaError_t err = attr_once.run(current_device(), [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem_bytes(1024));
+  });
+  if (err != cudaSuccess) return err;
   const long long max_tiles = ((long long)(p.S + BM2 - 1) / BM2 + p.E) * p.ntn;
   long long clusters = max_pair_clusters<GATEUP>(C::smem_bytes(1024));
   if (max_tiles < clusters) clusters = max_tiles > 0 ? max_tiles : 1;
@@ -495,7 +488,7 @@ cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& ta64, const CUt
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = MOE_PDL ? 2 : 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, kern, ta, ta64, tb0, tb1, p);
+  err = cudaLaunchKernelEx(&cfg, kern, ta, ta64, tb0, tb1, p);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
