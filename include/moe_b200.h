@@ -62,7 +62,7 @@ extern "C" {
 typedef enum moe_status {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1, /* rejected on the host, nothing enqueued */
-  MOE_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  MOE_ERR_UNSUPPORTED = 2, /* valid request the library does not implement */
   MOE_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
   MOE_ERR_DEVICE = 4,      /* the device flagged bad data (see moe_get_error) */
   MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out */
