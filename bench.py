@@ -168,6 +168,7 @@ def algorithmic(wl):
         "dispatch_bytes": wl.T * wl.H * b + S * wl.H * b + 12 * S,  # x read, x_disp write, ids/ranks/maps
         "combine_bytes": S * wl.H * b + wl.T * wl.H * b + 8 * S,  # y_disp read, y write, w + slot_to_row
         "route_bytes": wl.T * wl.E * 4 + wl.T * wl.k * 8,
+        "router_bytes": wl.T * wl.H * 2 + wl.E * wl.H * 2 + wl.T * wl.k * 8,  # x, W_r read; ids, w written
         "gateup_flops": 4.0 * S * wl.H * wl.I,
         "down_flops": 2.0 * S * wl.H * wl.I,
     }
@@ -353,8 +354,32 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     dc_stream_ms = a.elapsed_time(b) / n_pairs
     del sets, xs
+
+    # The router affinities fused with the top-k (moe_router_topk): logits = x W_r^T + bias on
+    # tensor cores, then route's selection; L2 flushed before each call.  Not part of the step
+    # above, which starts from given logits.
+    router_ms = None
+    if wl.dtype == "bf16" and wl.E <= 256:
+        from token_dispatch_combine_b200 import moe_router_topk
+        w_router = torch.from_numpy(np.ascontiguousarray(wl.router_weight().T)).to(dev).to(torch.bfloat16)
+        r_bias = torch.from_numpy(wl.router_bias().astype(np.float32)).to(dev) if wl.bias != "none" else None
+        r_ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+        r_w = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            moe_router_topk(x, w_router, wl.k, bias=r_bias, topk_ids=r_ids, topk_w=r_w)
+        rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in rev:
+            flush_and_hold()
+            a.record(stream)
+            moe_router_topk(x, w_router, wl.k, bias=r_bias, topk_ids=r_ids, topk_w=r_w)
+            b.record(stream)
+        torch.cuda.synchronize()
+        router_ms = sum(a.elapsed_time(b) for a, b in rev) / args.steps
+        del w_router, r_ids, r_w
     step_ms, dc_pair_ms, dc_stream_ms, *stage_max = max_over_ranks(
         [step_ms, dc_pair_ms, dc_stream_ms, *stage.tolist()], world)
+    if router_ms is not None:
+        router_ms = max_over_ranks([router_ms], world)[0]
 
     # End to end through the public API: every step copies its inputs (x, logits) from pinned
     # host memory to the device and its output y back, inside the timed region.
@@ -424,6 +449,12 @@ def run_ours(args, wl):
             "stage_timing": "per-stage CUDA events in a separate pass of the same steps (each stage boundary "
                             "adds event overhead); back_to_back: one event pair around dispatch+combine; stream: 20 dispatch+combine pairs over 4 buffer sets (>L2) under one event pair",
             "grouped_gemm_tflops": gemm_tflops, "grouped_gemm_frac_bf16": gemm_tflops / peak_tf,
+            **({} if router_ms is None else {
+                "router_topk_us": router_ms * 1e3,
+                "router_topk_gbs": alg["router_bytes"] / (router_ms * 1e-3) / 1e9,
+                "router_topk_frac_hbm": alg["router_bytes"] / (router_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "router_topk_timing": "moe_router_topk (logits = x W_r^T + bias, then top-k), L2 flushed, "
+                                      "events per call; bytes T*H*2 + E*H*2 + T*k*8"}),
             "ffn_tiling": "pair" if tiling == FFN_TILING_PAIR else "single",
         },
         "roofline": {

@@ -94,6 +94,23 @@ moe_status moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids
                      void* stream);
 
 /*
+ * moe_router_topk -- [NEURON] "Router Weights": every token is scored against
+ * all E experts, logits = x W_r^T (+ bias); then exactly moe_route on those
+ * logits.  The affinity matrix runs on tensor cores: bf16 products summed in
+ * float32 (order of the tensor-core accumulation), plus the bias in float32.
+ *   x        [T, H] bf16          token activations
+ *   w_router [E, H] bf16          row e = expert e's router vector
+ *   bias     [E] float32 or NULL  added to every token's logits
+ *   logits   [T, E] float32 or NULL  out (optional): the affinities used
+ *   topk_ids [T, k] int32, topk_w [T, k] float32  out: as moe_route, and
+ *            bit-identical to moe_route applied to the logits written here
+ * Constraints: T >= 0, 1 <= E <= 256, 1 <= k <= min(E, 8), H a positive
+ * multiple of 8; x, w_router 16-byte aligned.
+ */
+moe_status moe_router_topk(const void* x, const void* w_router, const float* bias, int T, int H, int E, int k,
+                           float* logits, int32_t* topk_ids, float* topk_w, void* stream);
+
+/*
  * Bytes of device workspace moe_dispatch needs for these sizes.  The
  * workspace must be zero-filled once before its first use; each call leaves
  * it ready for the next.  Calls sharing a workspace must not overlap.

@@ -48,6 +48,8 @@ def _configure(lib):
     lib.oracle_dispatch_rows.argtypes = [vp, sz, i32, i32, vp, vp]
     lib.oracle_ffn_rows.argtypes = [vp, i32, vp, i32, vp, vp, vp, i32, i32, i32, vp, vp]
     lib.oracle_combine.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+    lib.oracle_router_logits.argtypes = [vp, i32, vp, i32, vp, i32, i32, i32, vp]
+    lib.oracle_router_logits.restype = i32
     return lib
 
 
@@ -86,6 +88,25 @@ def route(logits: np.ndarray, k: int):
     if _get().oracle_route(logits.ctypes.data, T, E, k, ids.ctypes.data, w.ctypes.data) != 0:
         raise ValueError("oracle_route: bad sizes")
     return ids, w
+
+
+def router_logits(x: np.ndarray, w_router: np.ndarray, bias=None) -> np.ndarray:
+    """Affinities [T,E] float32 = round_f32(x @ w_router.T + bias) in float64.
+
+    ``x`` [T,H] and ``w_router`` [E,H] are float32 or bf16 bits (uint16);
+    ``bias`` [E] (any float type) or None."""
+    x = np.ascontiguousarray(x)
+    w = np.ascontiguousarray(w_router)
+    T, H = x.shape
+    E = w.shape[0]
+    if w.shape[1] != H:
+        raise ValueError("w_router must be [E, H]")
+    b = None if bias is None else _c(bias, np.float64)
+    out = np.empty((T, E), np.float32)
+    if _get().oracle_router_logits(x.ctypes.data, _dt(x), w.ctypes.data, _dt(w),
+                                   None if b is None else b.ctypes.data, T, H, E, out.ctypes.data) != 0:
+        raise ValueError("oracle_router_logits: bad sizes")
+    return out
 
 
 def src_rank(t: int, T: int, R: int) -> int:

@@ -51,6 +51,30 @@ static double orc_load(const void* base, int dtype, size_t i) {
   return (double)f;
 }
 
+/* ---------------------------------------------------------- router logits
+ * [NEURON] "Router Weights": every token is scored against all E experts;
+ * the affinity of token t for expert e is the dot product of the token's
+ * activation with expert e's router vector, plus the expert's bias:
+ *   logits[t][e] = round_f32( sum_h x[t][h] * w[e][h] + bias[e] )
+ * summed in float64 over ascending h from the given (bf16 or float32) values,
+ * rounded once to float32.  w is [E][H] (row e = expert e); bias may be NULL.
+ * Returns 0, or -1 for bad sizes.
+ */
+int oracle_router_logits(const void* x, int xdt, const void* w, int wdt, const double* bias, int T, int H, int E,
+                         float* logits) {
+  if (T < 0 || H < 1 || E < 1) return -1;
+  for (int t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += orc_load(x, xdt, (size_t)t * H + h) * orc_load(w, wdt, (size_t)e * H + h);
+      if (bias) acc += bias[e];
+      logits[(size_t)t * E + e] = (float)acc;
+    }
+  }
+  return 0;
+}
+
 /* ------------------------------------------------------------------ route
  * [EPRT] "Send tokens ...": the router chooses each token's expert(s) from
  * all E experts; Top-1 uses combination weight one.  "Return multiple ...":

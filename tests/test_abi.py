@@ -137,3 +137,27 @@ def test_library_override_variable_is_honoured(tmp_path):
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, check=True,
                          cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__)))).stdout.split()
     assert out[0] == str(copy) and int(out[1]) >= 1
+
+
+@pytest.mark.parametrize("kw,needle", [
+    (dict(E=257), b"E must be <= 256"),
+    (dict(H=60), b"multiple of 8"),
+    (dict(H=0), b"multiple of 8"),
+    (dict(k=9), b"k must"),
+    (dict(k=5, E=4), b"k must"),
+    (dict(T=-1), b"T must"),
+    (dict(x=FAKE + 8), b"x is not"),
+    (dict(bias=FAKE + 2), b"bias is not"),
+])
+def test_router_topk_rejects(kw, needle):
+    a = dict(x=FAKE, w=FAKE, bias=None, T=8, H=64, E=32, k=4, logits=None)
+    a.update(kw)
+    st = _native.lib().moe_router_topk(a["x"], a["w"], a["bias"], a["T"], a["H"], a["E"], a["k"], a["logits"],
+                                       FAKE, FAKE, None)
+    assert st == _native.MOE_ERR_INVALID_ARG
+    assert needle in _native.lib().moe_last_error_message()
+
+
+def test_router_topk_zero_tokens_is_a_host_no_op():
+    # T = 0 returns before any pointer is read or any launch
+    assert _native.lib().moe_router_topk(None, None, None, 0, 64, 32, 4, None, None, None, None) == 0

@@ -27,6 +27,8 @@ MUTANTS = {
     "round_robin_placement": ("for (int e = r * EL; e < (r + 1) * EL; ++e)", "for (int e = r; e < E; e += R)"),
     "src_rank_round_robin": ("(int)(((int64_t)t * R) / T)", "(t % R)"),
     "combine_ignores_weight": ("out[h] += wj * y_disp", "out[h] += y_disp"),
+    "router_weight_transposed": ("orc_load(w, wdt, (size_t)e * H + h)", "orc_load(w, wdt, (size_t)h * E + e)"),
+    "router_drops_bias": ("      if (bias) acc += bias[e];\n", "\n"),
     "combine_drops_last_choice": ("for (int j = 0; j < k; ++j) {\n      int row = slot_to_row", "for (int j = 0; j < k - 1; ++j) {\n      int row = slot_to_row"),
 }
 
@@ -43,6 +45,9 @@ PINS = [
     pins.test_swiglu_closed_forms,
     lambda: pins.test_round_trip_equals_dense_masked_moe(16, 32, 64, 8, 2, 4),
     pins.test_identity_experts_reproduce_input,
+    pins.test_router_logits_hand_example,
+    pins.test_router_logits_one_hot_rows_select_columns,
+    pins.test_router_logits_bias_only_and_bf16_widening,
 ]
 
 

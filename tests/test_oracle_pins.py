@@ -289,3 +289,50 @@ def test_identity_experts_reproduce_input():
             assert (y == x).all()
         else:
             np.testing.assert_allclose(y, x, rtol=0, atol=1e-6 * np.abs(x).max())
+
+
+# ---------------------------------------------------------------------------
+# Router affinities: "Expert Parallelism (EP)", "Router Weights" -- every token
+# scored against all E experts, logits = x W_r^T + bias.
+# ---------------------------------------------------------------------------
+def test_router_logits_hand_example():
+    # x = [[1, 2], [3, -1]], router rows e0 = (1, 0), e1 = (1, 1), e2 = (0, -2),
+    # bias (0.5, 0, -1): worked by hand
+    x = np.array([[1, 2], [3, -1]], np.float32)
+    w = np.array([[1, 0], [1, 1], [0, -2]], np.float32)
+    lg = oracle.router_logits(x, w, [0.5, 0.0, -1.0])
+    assert lg.tolist() == [[1.5, 3.0, -5.0], [3.5, 2.0, 1.0]]
+
+
+def test_router_logits_one_hot_rows_select_columns():
+    # a one-hot router row picks one activation column: catches transposed or
+    # shifted indices
+    rng = np.random.default_rng(3)
+    T, H, E = 7, 11, 5
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    cols = [4, 0, 10, 4, 7]
+    w = np.zeros((E, H), np.float32)
+    for e, c in enumerate(cols):
+        w[e, c] = 1.0
+    lg = oracle.router_logits(x, w)
+    assert (lg == x[:, cols]).all()
+
+
+def test_router_logits_bias_only_and_bf16_widening():
+    # zero activations give the bias; bf16 bits widen exactly (1.5, -2, 0.25)
+    lg = oracle.router_logits(np.zeros((2, 3), np.float32), np.ones((4, 3), np.float32), [1, -2, 0.25, 0])
+    assert lg.tolist() == [[1.0, -2.0, 0.25, 0.0]] * 2
+    xb = np.array([[0x3FC0, 0xC000, 0x3E80]], np.uint16)    # 1.5, -2, 0.25
+    wb = np.array([[0x3F80, 0x3F80, 0x4080]], np.uint16)    # 1, 1, 4
+    assert oracle.router_logits(xb, wb).tolist() == [[1.5 - 2.0 + 1.0]]
+
+
+def test_router_then_route_reproduces_worked_example():
+    # identity router (H = E): the logits are the activations, so routing the
+    # worked example's logits through the router gives the page's choices
+    g = _load("ep_worked_example.json")
+    x = np.array(g["logits"], np.float32)
+    lg = oracle.router_logits(x, np.eye(g["E"], dtype=np.float32))
+    ids, w = oracle.route(lg, g["k"])
+    assert ids.tolist() == g["expected"]["topk_ids"]
+    assert w.tolist() == g["expected"]["topk_w"]

@@ -22,7 +22,7 @@ ERR_BAD_ID, ERR_BAD_OFFSETS, ERR_BAD_ROW, ERR_TIMEOUT = 1, 2, 4, 8
 EXPORTS = (
     "moe_abi_version", "moe_status_string", "moe_last_error_message", "moe_route", "moe_dispatch_workspace_bytes",
     "moe_dispatch", "moe_expert_ffn", "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_get_error", "moe_selftest_wait_timeout",
-    "moe_dispatch_noalloc", "moe_set_ffn_tiling", "moe_get_ffn_tiling", "moe_ffn_tiling_for",
+    "moe_dispatch_noalloc", "moe_set_ffn_tiling", "moe_get_ffn_tiling", "moe_ffn_tiling_for", "moe_router_topk",
 )
 
 _lock = threading.Lock()
@@ -51,6 +51,7 @@ def _configure(lib):
         "moe_get_error": ([vp, u32p], i32),
         "moe_selftest_wait_timeout": ([ctypes.c_uint, vp], i32),
         "moe_dispatch_noalloc": ([vp, i32, i32, i32, vp, i32, i32, i32] + [vp] * 8 + [vp], i32),
+        "moe_router_topk": ([vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp], i32),
         "moe_set_ffn_tiling": ([i32], i32),
         "moe_get_ffn_tiling": ([], i32),
         "moe_ffn_tiling_for": ([i32, i32], i32),

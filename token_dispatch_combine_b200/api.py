@@ -54,6 +54,31 @@ def moe_route(logits: torch.Tensor, k: int, topk_ids: torch.Tensor | None = None
     return topk_ids, topk_w
 
 
+def moe_router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int, bias: torch.Tensor | None = None,
+                    topk_ids: torch.Tensor | None = None, topk_w: torch.Tensor | None = None,
+                    logits: torch.Tensor | None = None, want_logits: bool = False, stream=None):
+    """Router affinities x @ w_router.T (+ bias) on tensor cores, then the top-k
+    selection and softmax weights of ``moe_route`` on them, in one kernel.
+
+    x [T,H] bf16, w_router [E,H] bf16, bias [E] float32 or None.  Returns
+    (topk_ids [T,k] int32, topk_w [T,k] float32) and, when ``want_logits`` or
+    ``logits`` is given, the [T,E] float32 affinities as a third value."""
+    T, H = x.shape
+    E = w_router.shape[0]
+    dev = x.device
+    if topk_ids is None:
+        topk_ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if logits is None and want_logits:
+        logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    check(_native.lib().moe_router_topk(
+        _ptr(x, "x", torch.bfloat16), _ptr(w_router, "w_router", torch.bfloat16), _ptr(bias, "bias", torch.float32),
+        T, H, E, k, _ptr(logits, "logits", torch.float32), _ptr(topk_ids, "topk_ids", torch.int32),
+        _ptr(topk_w, "topk_w", torch.float32), _stream(stream)), "moe_router_topk")
+    return (topk_ids, topk_w, logits) if logits is not None else (topk_ids, topk_w)
+
+
 def moe_dispatch_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
     return int(_native.lib().moe_dispatch_workspace_bytes(T, k, E, R))
 

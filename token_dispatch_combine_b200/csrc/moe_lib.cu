@@ -15,6 +15,7 @@
 #include "ffn_tc.cuh"
 #include "ffn_tc2.cuh"
 #include "route.cuh"
+#include "router.cuh"
 
 namespace {
 
@@ -111,6 +112,24 @@ moe_status moe_route(const float* logits, int T, int E, int k, int32_t* topk_ids
   MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
   MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
   return cuda_status(moe::launch_route(logits, T, E, k, topk_ids, topk_w, (cudaStream_t)stream), "moe_route");
+}
+
+moe_status moe_router_topk(const void* x, const void* w_router, const float* bias, int T, int H, int E, int k,
+                           float* logits, int32_t* topk_ids, float* topk_w, void* stream) {
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  moe_status st = check_k_e(k, E);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(E <= 256, "moe_router_topk: E must be <= 256");
+  MOE_REQUIRE(H >= 8 && H % 8 == 0, "moe_router_topk: H must be a positive multiple of 8");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(x, 16, "x");
+  MOE_REQUIRE_PTR(w_router, 16, "w_router");
+  if (bias != nullptr) MOE_REQUIRE_PTR(bias, 4, "bias");
+  if (logits != nullptr) MOE_REQUIRE_PTR(logits, 4, "logits");
+  MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
+  MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
+  const moe::tc::RouterParams p{bias, T, H, E, k, logits, topk_ids, topk_w};
+  return cuda_status(moe::tc::launch_router(x, w_router, p, (cudaStream_t)stream), "moe_router_topk");
 }
 
 size_t moe_dispatch_workspace_bytes(int T, int k, int E, int R) {

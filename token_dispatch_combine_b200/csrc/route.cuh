@@ -5,10 +5,8 @@
 // scores; "Return multiple expert results to the same token": the weights
 // used at combine are kept apart from the choice.
 //
-// One warp per token.  Lane l holds logits l, l+32, l+64, ... (coalesced).
-// Each of the k rounds takes a warp-wide arg-max with two redux ops: the
-// largest order key, then the smallest expert id among lanes holding it, so
-// equal logits resolve to the lower id exactly as the sorted definition does.
+// One warp per token (warp_topk_softmax); lane l loads logits l, l+32, ...
+// (coalesced).
 #pragma once
 
 #include "common.cuh"
@@ -24,6 +22,50 @@ __device__ __forceinline__ uint32_t logit_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Top-k + softmax of one token by one warp.  Lane l holds the token's logits
+// l, l+32, l+64, ... (val[v] for expert l + 32 v; key[v] = logit_order_key, or
+// 0 for no expert).  Each of the k rounds takes a warp-wide arg-max with two
+// redux ops: the largest order key, then the smallest expert id among lanes
+// holding it, so equal logits resolve to the lower id.  Lane j < k gets the
+// j-th expert and its weight exp(l_j - l_0) / sum_i exp(l_i - l_0), the sum
+// taken in order i = 0..k-1.
+template <int VPL>
+__device__ __forceinline__ void warp_topk_softmax(uint32_t (&key)[VPL], const float (&val)[VPL], int k, int lane,
+                                                  int& my_id, float& my_w) {
+  my_id = 0;
+  float my_val = 0.0f;
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0;
+    int bid = 0x7FFFFFFF;
+    float bv = 0.0f;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      // ascending v visits ascending expert ids, so strict '>' keeps the lower id
+      const bool better = key[v] > bk;
+      bk = better ? key[v] : bk;
+      bid = better ? lane + 32 * v : bid;
+      bv = better ? val[v] : bv;
+    }
+    const uint32_t wk = __reduce_max_sync(0xFFFFFFFFu, bk);
+    const int wid = __reduce_min_sync(0xFFFFFFFFu, bk == wk ? bid : 0x7FFFFFFF);
+    const float wv = __shfl_sync(0xFFFFFFFFu, bv, wid & 31);  // the winner's logit, from its lane
+    const bool mine = (wid & 31) == lane;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) key[v] = (mine && v == (wid >> 5)) ? 0u : key[v];  // taken
+    if (lane == j) {
+      my_id = wid;
+      my_val = wv;
+    }
+  }
+  // softmax over the selected logits, max-subtracted (the first pick is the max)
+  const float l0 = __shfl_sync(0xFFFFFFFFu, my_val, 0);
+  const float ex = lane < k ? expf(my_val - l0) : 0.0f;
+  float sum = 0.0f;
+  for (int j = 0; j < k; ++j) sum += __shfl_sync(0xFFFFFFFFu, ex, j);  // fixed order j = 0..k-1
+  my_w = ex / sum;
+}
+
 template <int VPL>  // logits per lane: ceil(E / 32)
 __global__ void __launch_bounds__(256) route_topk_softmax_kernel(const float* __restrict__ logits, int T, int E,
                                                                  int k, int32_t* __restrict__ topk_ids,
@@ -36,44 +78,19 @@ __global__ void __launch_bounds__(256) route_topk_softmax_kernel(const float* __
   const float* row = logits + (size_t)t * E;
 
   uint32_t key[VPL];
+  float val[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) {
     const int e = lane + 32 * v;
-    key[v] = (e < E) ? logit_order_key(__ldg(row + e)) : 0u;
+    val[v] = (e < E) ? __ldg(row + e) : 0.0f;
+    key[v] = (e < E) ? logit_order_key(val[v]) : 0u;
   }
-
-  int my_id = 0;  // lane j keeps the j-th selected expert
-#pragma unroll 1
-  for (int j = 0; j < k; ++j) {
-    uint32_t bk = 0;
-    int bid = 0x7FFFFFFF;
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      // ascending v visits ascending expert ids, so strict '>' keeps the lower id
-      if (key[v] > bk) {
-        bk = key[v];
-        bid = lane + 32 * v;
-      }
-    }
-    const uint32_t wk = __reduce_max_sync(0xFFFFFFFFu, bk);
-    const int wid = __reduce_min_sync(0xFFFFFFFFu, bk == wk ? bid : 0x7FFFFFFF);
-    if ((wid & 31) == lane) {
-#pragma unroll
-      for (int v = 0; v < VPL; ++v)
-        if (v == (wid >> 5)) key[v] = 0u;  // taken
-    }
-    if (lane == j) my_id = wid;
-  }
-
-  // softmax over the selected logits, max-subtracted (the first pick is the max)
-  const float l0 = __shfl_sync(0xFFFFFFFFu, lane == 0 ? __ldg(row + my_id) : 0.0f, 0);
-  float ex = 0.0f;
-  if (lane < k) ex = expf(__ldg(row + my_id) - l0);
-  float sum = 0.0f;
-  for (int j = 0; j < k; ++j) sum += __shfl_sync(0xFFFFFFFFu, ex, j);  // fixed order j = 0..k-1
+  int my_id;
+  float my_w;
+  warp_topk_softmax<VPL>(key, val, k, lane, my_id, my_w);
   if (lane < k) {
     topk_ids[(size_t)t * k + lane] = my_id;
-    topk_w[(size_t)t * k + lane] = ex / sum;
+    topk_w[(size_t)t * k + lane] = my_w;
   }
 }
 
