@@ -240,8 +240,8 @@ def config_dict(wl):
 def run_ours(args, wl):
     import torch
 
-    from token_dispatch_combine_b200 import (FFN_TILING_PAIR, MoERoundTrip, moe_ffn_tiling_for, moe_get_error,
-                                             moe_set_ffn_tiling)
+    from token_dispatch_combine_b200 import (FFN_DOWN, FFN_GATE_UP, FFN_TILING_PAIR, MoERoundTrip, moe_ffn_tiling_for,
+                                             moe_get_error, moe_set_ffn_tiling)
     moe_set_ffn_tiling({"auto": 0, "single": 1, "pair": 2}[args.ffn_tiling])
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -255,7 +255,9 @@ def run_ours(args, wl):
 
     x, logits = up(x_np), up(logits_np)
     wg, wu, wd = up(wg_np), up(wu_np), up(wd_np)
-    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev)
+    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev,
+                      gather={"auto": "auto", "rows": False, "gather": True}[args.dispatch])
+    gather = rt.gather
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     flush_max = torch.empty((), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
@@ -323,26 +325,49 @@ def run_ours(args, wl):
         stage += [ev[j].elapsed_time(ev[j + 1]) for j in range(5)]
     stage /= args.steps  # ms per step per stage: route, dispatch, gate_up, down, combine
 
+    # The dispatch+combine metric is about the row-moving dispatch: when the step gathers its
+    # rows in the gate/up projection, measure dispatch (with rows) and combine on a second,
+    # row-moving round trip of the same layer.
+    if gather:
+        rt_dc = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev, gather=False)
+        rt_dc.forward(x, logits, wg, wu, wd)
+        dc_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        for ev in dc_ev:
+            flush_and_hold()
+            ev[0].record(stream)
+            rt_dc.dispatch(x)
+            ev[1].record(stream)
+            flush_and_hold()
+            ev[2].record(stream)
+            rt_dc.combine()
+            ev[3].record(stream)
+        torch.cuda.synchronize()
+        dc_stage = [sum(ev[0].elapsed_time(ev[1]) for ev in dc_ev) / args.steps,
+                    sum(ev[2].elapsed_time(ev[3]) for ev in dc_ev) / args.steps]
+    else:
+        rt_dc = rt
+        dc_stage = [float(stage[1]), float(stage[4])]
+
     # Dispatch and combine back to back (same bytes: combine reads the previous step's y_disp),
     # one event pair around both, L2 flushed before: their cost without the per-stage events.
     pair = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for a, b in pair:
         flush_and_hold()
         a.record(stream)
-        rt.dispatch(x)
-        rt.combine()
+        rt_dc.dispatch(x)
+        rt_dc.combine()
         b.record(stream)
     torch.cuda.synchronize()
     dc_pair_ms = sum(a.elapsed_time(b) for a, b in pair) / args.steps
     # Dispatch + combine as a stream of layers: 4 independent buffer sets (x, dispatched rows,
     # y_disp, y: ~1.3 GB, far beyond the 126 MB L2) visited in turn, 20 pairs under one event pair.
     # Launch latency is then overlapped as it is inside a step, and no pair finds its data in L2.
-    sets = [MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev) for _ in range(4)]
+    sets = [MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev, gather=False) for _ in range(4)]
     xs = [x.clone() for _ in sets]
     for r_, x_ in zip(sets, xs):
         r_.route(logits)
         r_.dispatch(x_)
-        r_.y_disp.copy_(rt.y_disp)
+        r_.y_disp.copy_(rt_dc.y_disp)
     n_pairs = 20
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     flush_and_hold()
@@ -354,6 +379,8 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     dc_stream_ms = a.elapsed_time(b) / n_pairs
     del sets, xs
+    if gather:
+        del rt_dc
 
     # The router affinities fused with the top-k (moe_router_topk): logits = x W_r^T + bias on
     # tensor cores, then route's selection; L2 flushed before each call.  Not part of the step
@@ -376,8 +403,8 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         router_ms = sum(a.elapsed_time(b) for a, b in rev) / args.steps
         del w_router, r_ids, r_w
-    step_ms, dc_pair_ms, dc_stream_ms, *stage_max = max_over_ranks(
-        [step_ms, dc_pair_ms, dc_stream_ms, *stage.tolist()], world)
+    step_ms, dc_pair_ms, dc_stream_ms, t_disp_rows, t_comb_rows, *stage_max = max_over_ranks(
+        [step_ms, dc_pair_ms, dc_stream_ms, *dc_stage, *stage.tolist()], world)
     if router_ms is not None:
         router_ms = max_over_ranks([router_ms], world)[0]
 
@@ -414,10 +441,11 @@ def run_ours(args, wl):
     alg = algorithmic(wl)
     t_route, t_disp, t_gu, t_down, t_comb = stage_max
     gemm_tflops = (alg["gateup_flops"] + alg["down_flops"]) / ((t_gu + t_down) * 1e-3) / 1e12
-    dc_gbs = (alg["dispatch_bytes"] + alg["combine_bytes"]) / ((t_disp + t_comb) * 1e-3) / 1e9
+    dc_gbs = (alg["dispatch_bytes"] + alg["combine_bytes"]) / ((t_disp_rows + t_comb_rows) * 1e-3) / 1e9
     gu_tflops = alg["gateup_flops"] / (t_gu * 1e-3) / 1e12
     peak_tf = peaks["bf16_tflops"]
-    tiling = moe_ffn_tiling_for(wl.E, wl.S)
+    tiling = moe_ffn_tiling_for(wl.E, wl.S, FFN_GATE_UP)
+    tiling_down = moe_ffn_tiling_for(wl.E, wl.S, FFN_DOWN)
     cpu = None
     if args.cpu_baseline and world == 1:
         rng = np.random.default_rng(1)
@@ -435,8 +463,11 @@ def run_ours(args, wl):
         "dtype": wl.dtype, "data": "synthetic",
         "config": config_dict(wl),
         "components": {
+            "dispatch_mode": ("index-only dispatch; the gate/up projection gathers its rows from x"
+                              if gather else "dispatch moves the rows into x_disp"),
             "route_us": t_route * 1e3, "dispatch_us": t_disp * 1e3, "gate_up_us": t_gu * 1e3,
             "down_us": t_down * 1e3, "combine_us": t_comb * 1e3,
+            "dispatch_rows_us": t_disp_rows * 1e3,
             "dispatch_combine_gbs": dc_gbs, "dispatch_combine_frac_hbm": dc_gbs / peaks["hbm_gbs"],
             "dispatch_combine_back_to_back_us": dc_pair_ms * 1e3,
             "dispatch_combine_back_to_back_gbs": (alg["dispatch_bytes"] + alg["combine_bytes"]) / (dc_pair_ms * 1e-3) / 1e9,
@@ -455,12 +486,15 @@ def run_ours(args, wl):
                 "router_topk_frac_hbm": alg["router_bytes"] / (router_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "router_topk_timing": "moe_router_topk (logits = x W_r^T + bias, then top-k), L2 flushed, "
                                       "events per call; bytes T*H*2 + E*H*2 + T*k*8"}),
-            "ffn_tiling": "pair" if tiling == FFN_TILING_PAIR else "single",
+            "ffn_tiling": {"gate_up": "pair" if tiling == FFN_TILING_PAIR else "single",
+                           "down": "pair" if tiling_down == FFN_TILING_PAIR else "single"},
         },
         "roofline": {
-            "kernel": ("grouped_gemm_tc2_kernel<gate/up, SwiGLU epilogue> (256-row tiles on 2-SM clusters)"
+            "kernel": ("grouped_gemm_tc2_kernel<gate/up, SwiGLU epilogue" + (", rows gathered from x" if gather else "")
+                       + "> (256-row tiles on 2-SM clusters)"
                        if tiling == FFN_TILING_PAIR else
-                       "grouped_gemm_tc_kernel<gate/up, SwiGLU epilogue> (128-row tiles)"),
+                       "grouped_gemm_tc_kernel<gate/up, SwiGLU epilogue" + (", rows gathered from x" if gather else "")
+                       + "> (128-row tiles)"),
             "bound": "tensor", "achieved": gu_tflops, "peak": peak_tf, "unit": "TFLOP/s",
             "frac": gu_tflops / peak_tf, "traffic": dram_traffic(wl.name),
             "peak_source": f"{peak_src} bf16 dense (burst)",
@@ -486,6 +520,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ffn-tiling", default="auto", choices=["auto", "single", "pair"],
                     help="tile shape of the bf16 expert FFN (moe_set_ffn_tiling); auto picks by rows per expert")
+    ap.add_argument("--dispatch", default="auto", choices=["auto", "rows", "gather"],
+                    help="rows: dispatch writes x_disp; gather: index-only dispatch, the gate/up projection "
+                         "gathers its rows from x (moe_ffn_gate_up_gather); auto: MoERoundTrip's choice")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false",
                     help="skip the CPU oracle leg (used for profiler runs)")
     args = ap.parse_args()

@@ -140,6 +140,10 @@ size_t moe_dispatch_workspace_bytes(int T, int k, int E, int R);
  * Rows are ordered by (expert, token): stable in token order within each
  * expert.  Slots with an id outside [0, E) are dropped (not counted,
  * slot_to_row = -1) and flagged in the device error word.
+ * Index-only dispatch: x and x_disp both NULL computes every output but
+ * x_disp (the counts, offsets and permutation) and moves no rows; the gate/up
+ * projection then gathers the rows itself (moe_ffn_gate_up_gather).  Exactly
+ * one of them NULL is MOE_ERR_INVALID_ARG.
  * Constraints: H * sizeof(dtype) % 16 == 0, E % R == 0, E <= 1024,
  * 1 <= k <= min(E, 8), S < 2^31.
  */
@@ -197,10 +201,12 @@ moe_status moe_expert_ffn(const void* x_disp, int dtype, const void* w_gate, con
 
 /*
  * Tile shape of the bf16 expert FFN (moe_expert_ffn, moe_ffn_gate_up,
- * moe_ffn_down).  One setting for the whole process, read at each call.
- *   MOE_FFN_TILING_AUTO    pair tiles when S >= 384 * E (enough rows per expert
- *                          that padding each expert to 256 rows costs little),
- *                          else single tiles.  The default.
+ * moe_ffn_down and their _gather forms).  One setting for the whole process,
+ * read at each call.
+ *   MOE_FFN_TILING_AUTO    per projection: pair tiles when S >= 448 * E for
+ *                          gate/up and S >= 384 * E for down (enough rows per
+ *                          expert that padding each expert to 256 rows costs
+ *                          little), else single tiles.  The default.
  *   MOE_FFN_TILING_SINGLE  128-row tiles, one SM per tile.
  *   MOE_FFN_TILING_PAIR    256-row tiles computed by a cluster of two SMs
  *                          (tcgen05 cta_group::2; each SM loads half of the
@@ -210,14 +216,17 @@ moe_status moe_expert_ffn(const void* x_disp, int dtype, const void* w_gate, con
  * same K order.  float32 calls ignore the setting.
  * moe_set_ffn_tiling returns MOE_ERR_INVALID_ARG for any other mode and keeps
  * the old one.  moe_ffn_tiling_for returns the shape (SINGLE or PAIR) that a
- * bf16 call with E experts and S rows would use now, or -1 for E <= 0 or S < 0.
+ * bf16 call of `projection` (MOE_FFN_GATE_UP or MOE_FFN_DOWN) with E experts
+ * and S rows would use now, or -1 for E <= 0, S < 0 or another projection.
  */
 #define MOE_FFN_TILING_AUTO 0
 #define MOE_FFN_TILING_SINGLE 1
 #define MOE_FFN_TILING_PAIR 2
+#define MOE_FFN_GATE_UP 0
+#define MOE_FFN_DOWN 1
 moe_status moe_set_ffn_tiling(int mode);
 int moe_get_ffn_tiling(void);
-int moe_ffn_tiling_for(int E, int S);
+int moe_ffn_tiling_for(int E, int S, int projection);
 
 /* First half of moe_expert_ffn: h = SiLU(x_disp Wg_e) * (x_disp Wu_e). */
 moe_status moe_ffn_gate_up(const void* x_disp, int dtype, const void* w_gate, const void* w_up,
@@ -226,6 +235,35 @@ moe_status moe_ffn_gate_up(const void* x_disp, int dtype, const void* w_gate, co
 /* Second half of moe_expert_ffn: y_disp = h Wd_e. */
 moe_status moe_ffn_down(const void* h, int dtype, const void* w_down, const int32_t* expert_offsets, int E, int H,
                         int I, int S, void* y_disp, void* stream);
+
+/*
+ * moe_ffn_gate_up_gather -- moe_ffn_gate_up fused with the row scatter of
+ * moe_dispatch ([EPRT] "Send tokens ...": a dispatched row is a copy of its
+ * token's row): the A operand of dispatched row r is read straight from x,
+ *   h[r] = SiLU(x[row_to_slot[r] / k] Wg_e) * (x[row_to_slot[r] / k] Wu_e),
+ * so x_disp is never written or read.  bf16: 128 extra threads per CTA copy
+ * each k-block's token rows into the swizzled A tile with 16-byte cp.async
+ * (the weights still arrive by TMA); float32 indexes x on CUDA cores.
+ * Measured against moe_dispatch + moe_ffn_gate_up: faster end to end where
+ * the FFN streams weights (few rows per expert), slower (~10% on the gate/up
+ * projection) where it is tensor-bound.
+ *   x              [T, H] dtype        token rows (moe_dispatch's x)
+ *   row_to_slot    [S] int32           from moe_dispatch (index-only is enough)
+ *   k              top-k of the routing (slot s belongs to token s / k)
+ *   the rest as moe_ffn_gate_up; S <= T * k.
+ * The result equals moe_ffn_gate_up on the x_disp that moe_dispatch writes,
+ * bit for bit (same products, same K order, same tile shape).  A row whose
+ * slot is outside [0, T * k) reads token 0 and is flagged (bit 4).
+ */
+moe_status moe_ffn_gate_up_gather(const void* x, int dtype, int T, const int32_t* row_to_slot, int k,
+                                  const void* w_gate, const void* w_up, const int32_t* expert_offsets, int E, int H,
+                                  int I, int S, void* h, void* stream);
+
+/* moe_expert_ffn with the gathering gate/up projection: moe_ffn_gate_up_gather, then moe_ffn_down. */
+moe_status moe_expert_ffn_gather(const void* x, int dtype, int T, const int32_t* row_to_slot, int k,
+                                 const void* w_gate, const void* w_up, const void* w_down,
+                                 const int32_t* expert_offsets, int E, int H, int I, int S, void* h, void* y_disp,
+                                 void* stream);
 
 /*
  * moe_combine -- [EPRT] "Send tokens ...": results return to their source

@@ -64,10 +64,10 @@ def test_route_rejects_misaligned_pointer():
 
 
 def _dispatch(**kw):
-    a = dict(x=FAKE, dtype=1, T=8, H=64, ids=FAKE, k=2, E=8, R=2, ws_bytes=1 << 20)
+    a = dict(x=FAKE, dtype=1, T=8, H=64, ids=FAKE, k=2, E=8, R=2, ws_bytes=1 << 20, x_disp=FAKE)
     a.update(kw)
-    return _native.lib().moe_dispatch(a["x"], a["dtype"], a["T"], a["H"], a["ids"], a["k"], a["E"], a["R"], FAKE,
-                                      FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, a["ws_bytes"], None)
+    return _native.lib().moe_dispatch(a["x"], a["dtype"], a["T"], a["H"], a["ids"], a["k"], a["E"], a["R"],
+                                      a["x_disp"], FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, a["ws_bytes"], None)
 
 
 @pytest.mark.parametrize("kw,needle", [
@@ -77,10 +77,38 @@ def _dispatch(**kw):
     (dict(k=3, E=2, R=1), b"k must"),
     (dict(ws_bytes=16), b"workspace_bytes"),
     (dict(x=FAKE + 8), b"x is not"),
+    (dict(x=None), b"both"),                       # index-only dispatch needs x and x_disp both NULL
+    (dict(x_disp=None), b"both"),
 ])
 def test_dispatch_rejects(kw, needle):
     assert _dispatch(**kw) == _native.MOE_ERR_INVALID_ARG
     assert needle in _native.lib().moe_last_error_message()
+
+
+@pytest.mark.parametrize("kw,needle", [
+    (dict(k=9), b"k must"),
+    (dict(S=17), b"S must be <= T * k"),
+    (dict(rts=FAKE + 2), b"row_to_slot"),
+    (dict(x=FAKE + 8), b"x is not"),
+    (dict(H=68), b"multiples of 16"),
+    (dict(T=-1), b"T must"),
+])
+def test_gate_up_gather_rejects(kw, needle):
+    a = dict(x=FAKE, dtype=1, T=8, rts=FAKE, k=2, E=4, H=64, I=64, S=16)
+    a.update(kw)
+    lib = _native.lib()
+    st = lib.moe_ffn_gate_up_gather(a["x"], a["dtype"], a["T"], a["rts"], a["k"], FAKE, FAKE, FAKE, a["E"], a["H"],
+                                    a["I"], a["S"], FAKE, None)
+    assert st == _native.MOE_ERR_INVALID_ARG
+    assert needle in lib.moe_last_error_message()
+    st = lib.moe_expert_ffn_gather(a["x"], a["dtype"], a["T"], a["rts"], a["k"], FAKE, FAKE, FAKE, FAKE, a["E"],
+                                   a["H"], a["I"], a["S"], FAKE, FAKE, None)
+    assert st == _native.MOE_ERR_INVALID_ARG
+
+
+def test_gate_up_gather_zero_rows_is_a_no_op():
+    # S = 0: validated, then nothing to launch (no device needed)
+    assert _native.lib().moe_ffn_gate_up_gather(FAKE, 1, 0, None, 2, None, None, FAKE, 4, 64, 64, 0, None, None) == 0
 
 
 def test_ffn_and_combine_reject():
@@ -104,17 +132,26 @@ def test_ffn_tiling_setting_is_host_only():
     lib = _native.lib()
     assert moe.moe_get_ffn_tiling() == moe.FFN_TILING_AUTO
     try:
-        # auto: pair tiles from 384 rows per expert on
-        assert moe.moe_ffn_tiling_for(32, 16384) == moe.FFN_TILING_PAIR
-        assert moe.moe_ffn_tiling_for(32, 384 * 32) == moe.FFN_TILING_PAIR
-        assert moe.moe_ffn_tiling_for(32, 384 * 32 - 1) == moe.FFN_TILING_SINGLE
-        assert moe.moe_ffn_tiling_for(256, 65536) == moe.FFN_TILING_SINGLE
+        # auto: pair tiles from 448 (gate/up) / 384 (down) rows per expert on
+        GU, DN = moe.FFN_GATE_UP, moe.FFN_DOWN
+        assert moe.moe_ffn_tiling_for(32, 16384) == moe.FFN_TILING_PAIR  # gate/up by default
+        assert moe.moe_ffn_tiling_for(32, 16384, DN) == moe.FFN_TILING_PAIR
+        assert moe.moe_ffn_tiling_for(32, 448 * 32, GU) == moe.FFN_TILING_PAIR
+        assert moe.moe_ffn_tiling_for(32, 448 * 32 - 1, GU) == moe.FFN_TILING_SINGLE
+        assert moe.moe_ffn_tiling_for(32, 384 * 32, DN) == moe.FFN_TILING_PAIR
+        assert moe.moe_ffn_tiling_for(32, 384 * 32 - 1, DN) == moe.FFN_TILING_SINGLE
+        assert moe.moe_ffn_tiling_for(32, 400 * 32, GU) == moe.FFN_TILING_SINGLE
+        assert moe.moe_ffn_tiling_for(32, 400 * 32, DN) == moe.FFN_TILING_PAIR
+        assert moe.moe_ffn_tiling_for(256, 65536, GU) == moe.FFN_TILING_SINGLE
+        assert moe.moe_ffn_tiling_for(256, 65536, DN) == moe.FFN_TILING_SINGLE
         assert moe.moe_ffn_tiling_for(0, 10) == -1
+        assert moe.moe_ffn_tiling_for(32, 10, 2) == -1
         for mode in (moe.FFN_TILING_SINGLE, moe.FFN_TILING_PAIR):
             moe.moe_set_ffn_tiling(mode)
             assert moe.moe_get_ffn_tiling() == mode
-            assert moe.moe_ffn_tiling_for(256, 1) == mode
-            assert moe.moe_ffn_tiling_for(1, 1 << 20) == mode
+            for proj in (GU, DN):
+                assert moe.moe_ffn_tiling_for(256, 1, proj) == mode
+                assert moe.moe_ffn_tiling_for(1, 1 << 20, proj) == mode
         assert lib.moe_set_ffn_tiling(3) == _native.MOE_ERR_INVALID_ARG
         assert lib.moe_set_ffn_tiling(-1) == _native.MOE_ERR_INVALID_ARG
         assert moe.moe_get_ffn_tiling() == moe.FFN_TILING_PAIR  # unchanged by the rejected calls

@@ -1,5 +1,10 @@
 """GPU round trip (through the C ABI) against the CPU oracle.
 
+These tests run the row-moving dispatch (x_disp is checked against the
+oracle's); the dispatch fused into the gate/up projection is checked in
+test_gpu_gather.py, and the host-pipeline and graph tests below run the
+round trip's default choice between the two.
+
 Integer outputs (ids, counts, offsets, permutation, dispatched rows) must be
 bit-exact; combination weights within 1e-6; float outputs within the
 normwise bound max|gpu - oracle| / max|oracle| <= 1e-4 (float32 layers) or
@@ -41,7 +46,7 @@ def run_gpu(layer: DeviceLayer, rt=None):
     from token_dispatch_combine_b200 import MoERoundTrip, moe_get_error
     wl = layer.wl
     if rt is None:
-        rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, layer.x_dev.dtype)
+        rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, layer.x_dev.dtype, gather=False)
     rt.forward(layer.x_dev, layer.logits_dev, layer.w_gate, layer.w_up, layer.w_down)
     st, bits = moe_get_error()
     assert st == 0 and bits == 0, (st, bits)
@@ -142,7 +147,8 @@ def test_single_and_pair_tiles_agree_bit_for_bit():
         try:
             for mode in (1, 2):
                 moe_set_ffn_tiling(mode)
-                rt = run_gpu(layer, MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, layer.x_dev.dtype))
+                rt = run_gpu(layer, MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, layer.x_dev.dtype,
+                                                 gather=False))
                 outs.append([t.view(torch.int16).clone() for t in (rt.h, rt.y_disp, rt.y)])
         finally:
             moe_set_ffn_tiling(0)
@@ -184,7 +190,7 @@ def test_identity_experts_combine_reproduces_input():
     from token_dispatch_combine_b200 import MoERoundTrip, moe_combine
     wl = W("ident", T=200, H=64, I=64, E=8, k=4, R=4, dtype="f32", seed=18)
     layer = DeviceLayer(wl)
-    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, torch.float32)
+    rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, torch.float32, gather=False)
     rt.route(layer.logits_dev)
     rt.dispatch(layer.x_dev)
     y = torch.empty_like(layer.x_dev)

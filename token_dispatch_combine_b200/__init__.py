@@ -7,16 +7,18 @@ the same names (``api``).  Importing it builds/loads the library and raises
 if that is impossible: there is no other implementation to fall back to.
 """
 from . import _native
-from .api import (DispatchOut, MoEHostPipeline, MoERoundTrip, moe_combine, moe_dispatch, moe_dispatch_workspace_bytes, moe_expert_ffn,
-                  moe_ffn_down, moe_ffn_gate_up, moe_ffn_tiling_for, moe_get_error, moe_get_ffn_tiling, moe_route,
-                  moe_router_topk, moe_set_ffn_tiling, new_dispatch_workspace)
-from ._native import FFN_TILING_AUTO, FFN_TILING_PAIR, FFN_TILING_SINGLE, MoeError
+from .api import (DispatchOut, MoEHostPipeline, MoERoundTrip, moe_combine, moe_dispatch, moe_dispatch_workspace_bytes,
+                  moe_expert_ffn, moe_expert_ffn_gather, moe_ffn_down, moe_ffn_gate_up, moe_ffn_gate_up_gather,
+                  moe_ffn_tiling_for, moe_get_error, moe_get_ffn_tiling, moe_route, moe_router_topk,
+                  moe_set_ffn_tiling, new_dispatch_workspace)
+from ._native import FFN_DOWN, FFN_GATE_UP, FFN_TILING_AUTO, FFN_TILING_PAIR, FFN_TILING_SINGLE, MoeError
 
 _native.lib()  # build (if needed) and load now: fail loudly at import
 
 __all__ = [
     "DispatchOut", "MoEHostPipeline", "MoERoundTrip", "MoeError", "moe_combine", "moe_dispatch", "moe_dispatch_workspace_bytes",
-    "moe_expert_ffn", "moe_ffn_down", "moe_ffn_gate_up", "moe_get_error", "moe_route", "new_dispatch_workspace",
-    "moe_set_ffn_tiling", "moe_get_ffn_tiling", "moe_ffn_tiling_for", "FFN_TILING_AUTO", "FFN_TILING_SINGLE",
-    "FFN_TILING_PAIR", "moe_router_topk",
+    "moe_expert_ffn", "moe_expert_ffn_gather", "moe_ffn_down", "moe_ffn_gate_up", "moe_ffn_gate_up_gather",
+    "moe_get_error", "moe_route", "new_dispatch_workspace", "moe_set_ffn_tiling", "moe_get_ffn_tiling",
+    "moe_ffn_tiling_for", "FFN_TILING_AUTO", "FFN_TILING_SINGLE", "FFN_TILING_PAIR", "FFN_GATE_UP", "FFN_DOWN",
+    "moe_router_topk",
 ]

@@ -15,6 +15,7 @@ from . import build as _build
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT = range(6)
 MOE_F32, MOE_BF16 = 0, 1
 FFN_TILING_AUTO, FFN_TILING_SINGLE, FFN_TILING_PAIR = 0, 1, 2
+FFN_GATE_UP, FFN_DOWN = 0, 1
 
 # error-word bits reported by moe_get_error
 ERR_BAD_ID, ERR_BAD_OFFSETS, ERR_BAD_ROW, ERR_TIMEOUT = 1, 2, 4, 8
@@ -23,6 +24,7 @@ EXPORTS = (
     "moe_abi_version", "moe_status_string", "moe_last_error_message", "moe_route", "moe_dispatch_workspace_bytes",
     "moe_dispatch", "moe_expert_ffn", "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_get_error", "moe_selftest_wait_timeout",
     "moe_dispatch_noalloc", "moe_set_ffn_tiling", "moe_get_ffn_tiling", "moe_ffn_tiling_for", "moe_router_topk",
+    "moe_ffn_gate_up_gather", "moe_expert_ffn_gather",
 )
 
 _lock = threading.Lock()
@@ -54,7 +56,9 @@ def _configure(lib):
         "moe_router_topk": ([vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp], i32),
         "moe_set_ffn_tiling": ([i32], i32),
         "moe_get_ffn_tiling": ([], i32),
-        "moe_ffn_tiling_for": ([i32, i32], i32),
+        "moe_ffn_tiling_for": ([i32, i32, i32], i32),
+        "moe_ffn_gate_up_gather": ([vp, i32, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp], i32),
+        "moe_expert_ffn_gather": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp], i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)

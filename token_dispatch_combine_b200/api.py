@@ -12,7 +12,7 @@ from dataclasses import dataclass
 import torch
 
 from . import _native
-from ._native import MOE_BF16, MOE_F32, check
+from ._native import FFN_GATE_UP, MOE_BF16, MOE_F32, check
 
 _DT = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}
 
@@ -85,7 +85,7 @@ def moe_dispatch_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
 
 @dataclass
 class DispatchOut:
-    x_disp: torch.Tensor
+    x_disp: torch.Tensor | None  # None: index-only dispatch (the gate/up projection gathers from x)
     expert_counts: torch.Tensor
     expert_offsets: torch.Tensor
     rank_counts: torch.Tensor
@@ -95,11 +95,11 @@ class DispatchOut:
     src_expert_counts: torch.Tensor | None
 
     @staticmethod
-    def empty(T, H, k, E, R, dtype, device, src_counts=True) -> "DispatchOut":
+    def empty(T, H, k, E, R, dtype, device, src_counts=True, rows=True) -> "DispatchOut":
         S = T * k
         i32 = dict(dtype=torch.int32, device=device)
         return DispatchOut(
-            x_disp=torch.empty((S, H), dtype=dtype, device=device),
+            x_disp=torch.empty((S, H), dtype=dtype, device=device) if rows else None,
             expert_counts=torch.empty(E, **i32), expert_offsets=torch.empty(E + 1, **i32),
             rank_counts=torch.empty(R, **i32), rank_offsets=torch.empty(R + 1, **i32),
             slot_to_row=torch.empty(S, **i32), row_to_slot=torch.empty(S, **i32),
@@ -111,13 +111,22 @@ def new_dispatch_workspace(T: int, k: int, E: int, R: int, device) -> torch.Tens
     return torch.zeros(moe_dispatch_workspace_bytes(T, k, E, R), dtype=torch.uint8, device=device)
 
 
-def moe_dispatch(x: torch.Tensor, topk_ids: torch.Tensor, E: int, R: int, out: DispatchOut, workspace: torch.Tensor,
-                 stream=None) -> DispatchOut:
-    T, H = x.shape
+def moe_dispatch(x: torch.Tensor | None, topk_ids: torch.Tensor, E: int, R: int, out: DispatchOut,
+                 workspace: torch.Tensor, stream=None, H: int | None = None, dtype=None) -> DispatchOut:
+    """Dispatch; with x None and out.x_disp None it is index-only (counts,
+    offsets and permutation; no rows move), and H / dtype name the row shape."""
+    if x is not None:
+        T, H = x.shape
+        dtype = x.dtype
+    else:
+        T = topk_ids.shape[0]
+        if H is None or dtype is None:
+            raise ValueError("index-only dispatch needs H and dtype")
     k = topk_ids.shape[1]
     i32 = torch.int32
     check(_native.lib().moe_dispatch(
-        _ptr(x, "x"), _dtype(x), T, H, _ptr(topk_ids, "topk_ids", i32), k, E, R, _ptr(out.x_disp, "x_disp", x.dtype),
+        _ptr(x, "x"), _DT[dtype] if dtype in _DT else _dtype(x), T, H, _ptr(topk_ids, "topk_ids", i32), k, E, R,
+        _ptr(out.x_disp, "x_disp", dtype),
         _ptr(out.expert_counts, "expert_counts", i32), _ptr(out.expert_offsets, "expert_offsets", i32),
         _ptr(out.rank_counts, "rank_counts", i32), _ptr(out.rank_offsets, "rank_offsets", i32),
         _ptr(out.slot_to_row, "slot_to_row", i32), _ptr(out.row_to_slot, "row_to_slot", i32),
@@ -142,6 +151,32 @@ def moe_ffn_down(h, w_down, expert_offsets, y_disp, stream=None):
     check(_native.lib().moe_ffn_down(
         _ptr(h, "h"), _dtype(h), _ptr(w_down, "w_down", h.dtype), _ptr(expert_offsets, "expert_offsets", torch.int32),
         E, H, I, S, _ptr(y_disp, "y_disp", h.dtype), _stream(stream)), "moe_ffn_down")
+    return y_disp
+
+
+def moe_ffn_gate_up_gather(x, row_to_slot, k, w_gate, w_up, expert_offsets, h, stream=None):
+    """h = SiLU(x[row_to_slot // k] Wg_e) * (x[row_to_slot // k] Wu_e): the gate/up
+    projection reading its rows straight from x (no x_disp)."""
+    T, H = x.shape
+    S = row_to_slot.shape[0]
+    E, _, I = w_gate.shape
+    dt = x.dtype
+    check(_native.lib().moe_ffn_gate_up_gather(
+        _ptr(x, "x"), _dtype(x), T, _ptr(row_to_slot, "row_to_slot", torch.int32), int(k), _ptr(w_gate, "w_gate", dt),
+        _ptr(w_up, "w_up", dt), _ptr(expert_offsets, "expert_offsets", torch.int32), E, H, I, S, _ptr(h, "h", dt),
+        _stream(stream)), "moe_ffn_gate_up_gather")
+    return h
+
+
+def moe_expert_ffn_gather(x, row_to_slot, k, w_gate, w_up, w_down, expert_offsets, h, y_disp, stream=None):
+    T, H = x.shape
+    S = row_to_slot.shape[0]
+    E, _, I = w_gate.shape
+    dt = x.dtype
+    check(_native.lib().moe_expert_ffn_gather(
+        _ptr(x, "x"), _dtype(x), T, _ptr(row_to_slot, "row_to_slot", torch.int32), int(k), _ptr(w_gate, "w_gate", dt),
+        _ptr(w_up, "w_up", dt), _ptr(w_down, "w_down", dt), _ptr(expert_offsets, "expert_offsets", torch.int32),
+        E, H, I, S, _ptr(h, "h", dt), _ptr(y_disp, "y_disp", dt), _stream(stream)), "moe_expert_ffn_gather")
     return y_disp
 
 
@@ -176,9 +211,10 @@ def moe_get_ffn_tiling() -> int:
     return _native.lib().moe_get_ffn_tiling()
 
 
-def moe_ffn_tiling_for(E: int, S: int) -> int:
-    """The tile shape (SINGLE or PAIR) a bf16 FFN call with E experts and S rows would use now."""
-    return _native.lib().moe_ffn_tiling_for(int(E), int(S))
+def moe_ffn_tiling_for(E: int, S: int, projection: int = FFN_GATE_UP) -> int:
+    """The tile shape (SINGLE or PAIR) a bf16 call of one projection
+    (FFN_GATE_UP or FFN_DOWN) with E experts and S rows would use now."""
+    return _native.lib().moe_ffn_tiling_for(int(E), int(S), int(projection))
 
 
 def moe_get_error(stream=None) -> tuple[int, int]:
@@ -195,16 +231,31 @@ class MoERoundTrip:
     Device memory for every intermediate is allocated once here (through
     torch); ``forward`` enqueues five kernels (route, dispatch, gate/up, down,
     combine) and allocates nothing.
+
+    gather=True fuses the row scatter into the gate/up projection: dispatch
+    is index-only and moe_ffn_gate_up_gather reads each row from x, so the
+    [S, H] x_disp buffer is neither allocated nor written (same results, bit
+    for bit).  gather="auto" (the default) fuses where that is measured to be
+    faster: bf16 layers with fewer than GATHER_MAX_ROWS_PER_EXPERT rows per
+    expert, whose FFN streams weights from HBM, so the x_disp round trip is
+    extra HBM traffic.  With more rows per expert the FFN is tensor-bound and
+    the gathering producer costs more than the dispatch it saves.
     """
 
-    def __init__(self, T, H, I, E, k, R, dtype, device="cuda", src_counts=True):
+    GATHER_MAX_ROWS_PER_EXPERT = 384
+
+    def __init__(self, T, H, I, E, k, R, dtype, device="cuda", src_counts=True, gather="auto"):
         self.T, self.H, self.I, self.E, self.k, self.R = T, H, I, E, k, R
         self.dtype = dtype
         self.device = torch.device(device)
+        if gather == "auto":
+            gather = dtype == torch.bfloat16 and T * k < self.GATHER_MAX_ROWS_PER_EXPERT * E
+        self.gather = bool(gather)
+        self._x = None
         S = T * k
         self.topk_ids = torch.empty((T, k), dtype=torch.int32, device=self.device)
         self.topk_w = torch.empty((T, k), dtype=torch.float32, device=self.device)
-        self.disp = DispatchOut.empty(T, H, k, E, R, dtype, self.device, src_counts)
+        self.disp = DispatchOut.empty(T, H, k, E, R, dtype, self.device, src_counts, rows=not self.gather)
         self.workspace = new_dispatch_workspace(T, k, E, R, self.device)
         self.h = torch.empty((S, I), dtype=dtype, device=self.device)
         self.y_disp = torch.empty((S, H), dtype=dtype, device=self.device)
@@ -214,9 +265,18 @@ class MoERoundTrip:
         return moe_route(logits, self.k, self.topk_ids, self.topk_w, stream)
 
     def dispatch(self, x, stream=None):
+        if self.gather:  # the rows stay in x; gate_up reads them there
+            self._x = x
+            return moe_dispatch(None, self.topk_ids, self.E, self.R, self.disp, self.workspace, stream,
+                                H=self.H, dtype=self.dtype)
         return moe_dispatch(x, self.topk_ids, self.E, self.R, self.disp, self.workspace, stream)
 
     def gate_up(self, w_gate, w_up, stream=None):
+        if self.gather:
+            if self._x is None:
+                raise RuntimeError("gate_up of a gathering round trip needs dispatch(x) first")
+            return moe_ffn_gate_up_gather(self._x, self.disp.row_to_slot, self.k, w_gate, w_up,
+                                          self.disp.expert_offsets, self.h, stream)
         return moe_ffn_gate_up(self.disp.x_disp, w_gate, w_up, self.disp.expert_offsets, self.h, stream)
 
     def down(self, w_down, stream=None):

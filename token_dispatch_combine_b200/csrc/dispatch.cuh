@@ -28,6 +28,8 @@
 //     16-byte vector accesses.  Before phase 1 each CTA asks L2 for its token
 //     rows of x and each warp loads its first slice, so those reads overlap
 //     the counting and the barriers.
+// With x_disp == nullptr (index-only dispatch, for a gate/up GEMM that gathers
+// its rows from x itself) phase 3 writes only the permutation.
 // A barrier that does not complete within 1 s sets the timeout bit of the
 // device error word; the kernel then returns without writing the rows.
 #pragma once
@@ -184,7 +186,8 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
   constexpr int N = Vec16<T>::N;
   const int nvec = H / N;
   const int tb = min(g.T, (int)blockIdx.x * tpc), te = min(g.T, tb + tpc);
-  if (threadIdx.x == 0 && te > tb) {
+  const bool copy_rows = x_disp != nullptr;  // index-only dispatch leaves the rows where they are
+  if (copy_rows && threadIdx.x == 0 && te > tb) {
     const char* base = reinterpret_cast<const char*>(x + (size_t)tb * H);
     const size_t bytes = (size_t)(te - tb) * H * sizeof(T);  // a multiple of 16 (H * sizeof(T) is)
     for (size_t b = 0; b < bytes; b += 65536) {
@@ -204,7 +207,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
   // ---- each warp's first slice of x into registers (it does not depend on the counts)
   uint4 pre[kScatterVecsPerLane];
   const int pre_tok = tb + warp / nslices, pre_cs = warp % nslices;
-  if (pre_tok < min(te, tb + kRowRound)) {
+  if (copy_rows && pre_tok < min(te, tb + kRowRound)) {
     const char* src = reinterpret_cast<const char*>(x + (size_t)pre_tok * H);
 #pragma unroll
     for (int u = 0; u < kScatterVecsPerLane; ++u) {
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
       if (row >= 0) row_to_slot[row] = s;
     }
     __syncthreads();
-    const int nit = (r1 - r0) * nslices;
+    const int nit = copy_rows ? (r1 - r0) * nslices : 0;
     for (int item = warp; item < nit; item += kDispatchWarps) {
       const int tl = item / nslices, cs = item - tl * nslices;
       uint4 v[kScatterVecsPerLane];
@@ -413,8 +416,10 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   const int nvec = H / Vec16<T>::N;
   const int nslices = (nvec + kScatterSlice - 1) / kScatterSlice;
   // phase 3: a CTA takes a contiguous token range; as many CTAs as keep every
-  // warp at one (token, slice) item, within the co-residency bound
-  const int tpc_one = kDispatchWarps / nslices > 0 ? kDispatchWarps / nslices : 1;
+  // warp at one (token, slice) item, within the co-residency bound (index
+  // only: one round of kRowRound tokens per CTA)
+  int tpc_one = kDispatchWarps / nslices > 0 ? kDispatchWarps / nslices : 1;
+  if (x_disp == nullptr) tpc_one = kRowRound;
   const long long item_ctas = ((long long)g.T + tpc_one - 1) / tpc_one;
   long long want = item_ctas > g.nchunks ? item_ctas : (long long)g.nchunks;
   if (want < 1) want = 1;

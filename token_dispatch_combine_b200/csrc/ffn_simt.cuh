@@ -31,12 +31,16 @@ __device__ __forceinline__ void expert_segment(const int32_t* __restrict__ off, 
   hi = b;
 }
 
+// gather != nullptr (gate/up only): A row r is row gather[r] / gk of A [gT, K]
+// (the token's row of x) instead of row r.
 template <typename T, bool GATEUP>
 __global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A, const T* __restrict__ B0,
                                                        const T* __restrict__ B1, const int32_t* __restrict__ off,
-                                                       int E, int K, int N, int S, T* __restrict__ out) {
+                                                       int E, int K, int N, int S, T* __restrict__ out,
+                                                       const int32_t* __restrict__ gather, int gk, int gT) {
   constexpr int BM = 64, BN = 64, BK = 16;
   __shared__ float As[BK][BM + 4];
+  __shared__ int s_src[BM];  // source row of A for each tile row (-1: none)
   __shared__ float Bs0[BK][BN];
   __shared__ float Bs1[GATEUP ? BK : 1][GATEUP ? BN : 1];
 
@@ -67,12 +71,26 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const T* __restrict__ A, 
 
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16 threads, 4 x 4 outputs each
   float acc0[4][4] = {}, acc1[4][4] = {};
+  if (threadIdx.x < BM) {
+    const int row = row0 + (int)threadIdx.x;
+    int src = row < row_end ? row : -1;
+    if (gather != nullptr && src >= 0) {
+      const int sl = __ldg(gather + row);
+      src = sl / gk;
+      if (sl < 0 || src >= gT) {
+        flag_error(kErrBadRow);
+        src = -1;
+      }
+    }
+    s_src[threadIdx.x] = src;
+  }
+  __syncthreads();
 
   for (int k0 = 0; k0 < K; k0 += BK) {
     for (int i = threadIdx.x; i < BM * BK; i += 256) {
       const int r = i / BK, kk = i % BK;
-      const int row = row0 + r, kx = k0 + kk;
-      As[kk][r] = (row < row_end && kx < K) ? (float)A[(size_t)row * K + kx] : 0.0f;
+      const int src = s_src[r], kx = k0 + kk;
+      As[kk][r] = (src >= 0 && kx < K) ? (float)A[(size_t)src * K + kx] : 0.0f;
     }
     for (int i = threadIdx.x; i < BK * BN; i += 256) {
       const int kk = i / BN, c = i % BN;
@@ -122,7 +140,21 @@ cudaError_t launch_ffn_simt_gate_up(const T* x_disp, const T* wg, const T* wu, c
   const int max_mtiles = (S + 63) / 64 + E;  // bound on sum_e ceil(count_e / 64)
   if (S == 0) return cudaSuccess;
   dim3 grid(max_mtiles, (I + 63) / 64);
-  cudaError_t err = launch_pdl(ffn_simt_kernel<T, true>, grid, 256, 0, stream, x_disp, wg, wu, off, E, H, I, S, h);
+  cudaError_t err = launch_pdl(ffn_simt_kernel<T, true>, grid, 256, 0, stream, x_disp, wg, wu, off, E, H, I, S, h,
+                               (const int32_t*)nullptr, 1, 0);
+  return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+// launch_ffn_simt_gate_up with the A rows gathered from x [T, H] by row_to_slot / k.
+template <typename T>
+cudaError_t launch_ffn_simt_gate_up_gather(const T* x, int T_, const int32_t* row_to_slot, int k, const T* wg,
+                                           const T* wu, const int32_t* off, int E, int H, int I, int S, T* h,
+                                           cudaStream_t stream) {
+  const int max_mtiles = (S + 63) / 64 + E;
+  if (S == 0) return cudaSuccess;
+  dim3 grid(max_mtiles, (I + 63) / 64);
+  cudaError_t err = launch_pdl(ffn_simt_kernel<T, true>, grid, 256, 0, stream, x, wg, wu, off, E, H, I, S, h,
+                               row_to_slot, k, T_);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
@@ -133,7 +165,7 @@ cudaError_t launch_ffn_simt_down(const T* h, const T* wd, const int32_t* off, in
   if (S == 0) return cudaSuccess;
   dim3 grid(max_mtiles, (H + 63) / 64);
   cudaError_t err = launch_pdl(ffn_simt_kernel<T, false>, grid, 256, 0, stream, h, wd, (const T*)nullptr, off, E, I,
-                               H, S, y);
+                               H, S, y, (const int32_t*)nullptr, 1, 0);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

@@ -31,6 +31,14 @@
 // 128 up columns side by side, so one N=256 MMA produces both halves of a
 // 128-column h tile in one accumulator.
 //
+// Gathering form (gate/up only, moe_ffn_gate_up_gather): the A rows are not
+// read from a dispatched buffer but copied from the token rows of x by 128
+// extra threads (warps 6..9) with 16-byte cp.async into the same swizzled
+// layout; each stage's full barrier then also counts one cp.async arrival
+// per gather thread, and the MMA thread fences the proxy before reading.
+// (TMA tile::gather4, four 128-byte rows per instruction, was measured first:
+// 32 instructions per k-block made the kernel 2.5-3x slower.)
+//
 // Every mbarrier wait is bounded (globaltimer): on expiry the CTA sets the
 // timeout bit of the device error word, the other roles stop, in-flight TMA
 // loads and MMAs are waited for (bounded), TMEM is freed and the kernel
@@ -61,6 +69,12 @@
 //    epilogue warp q holds rows 16q..16q+15 in its lanes 0-15.
 #ifndef MOE_TC_M64
 #define MOE_TC_M64 1
+#endif
+//  MOE_TC_GATHER_FENCE: the MMA thread of a gathering kernel issues a
+//    shared-memory proxy fence after each stage's full barrier, before its
+//    UMMAs read the rows that cp.async wrote.
+#ifndef MOE_TC_GATHER_FENCE
+#define MOE_TC_GATHER_FENCE 1
 #endif
 //  MOE_TC_DOWN_BN: force the down-projection n-tile width (0 = chosen from H).
 #ifndef MOE_TC_DOWN_BN
@@ -136,6 +150,23 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "[%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+// 16-byte global -> shared copy on the LSU path (cp.async); src_bytes = 0
+// writes 16 zero bytes and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrive on the mbarrier once all earlier cp.async of this thread have landed
+// (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Order shared-memory data made visible to this thread (written through the
+// generic proxy, e.g. by cp.async) before its later async-proxy accesses
+// (tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 // L2 eviction-priority policy for cache-hinted TMA loads (1 evict-first, 2 evict-last).
 template <int HINT>
@@ -232,7 +263,90 @@ struct Params {
   int E, S, K, N;          // N: output columns (I for gate/up, H for down)
   int ntn;                 // n-tiles per m-tile
   __nv_bfloat16* out;      // [S, N]
+  // Gathering kernels only: A row r is token row row_to_slot[r] / gather_k of
+  // x [gather_T, K] instead of row r of a dispatched buffer.
+  const int32_t* gather_rows;  // [S] row_to_slot
+  int gather_k, gather_T;
+  const void* gather_x;        // [gather_T, K] bf16
 };
+
+// ---- A-row gather (dispatch fused into the gate/up projection)
+// kGatherThreads extra threads per CTA copy the A tile rows of each k-block
+// from x with 16-byte cp.async: thread t owns 16-byte chunk c = t % 8 of rows
+// t / 8 + 16 j (j < 8) of the 128-row tile, written to its 128-byte
+// swizzled position (chunk c ^ (row % 8)).  Each thread then arrives on the
+// stage's full barrier when its copies land (cp.async.mbarrier.arrive.noinc).
+constexpr int kGatherThreads = 128;
+constexpr int kGatherRowsPerThread = 8;
+
+// Slots (row_to_slot entries) of this thread's rows of the tile [r0, r_end),
+// -1 for rows past r_end.  Loaded one tile ahead, so their latency hides
+// behind the previous tile's k-blocks.
+__device__ __forceinline__ void gather_load_slots(const Params& p, int r0, int r_end, int gt,
+                                                  int (&slot)[kGatherRowsPerThread]) {
+  const int rr = gt >> 3;
+#pragma unroll
+  for (int j = 0; j < kGatherRowsPerThread; ++j) {
+    const int r = r0 + rr + 16 * j;
+    slot[j] = r < r_end ? __ldg(p.gather_rows + r) : -1;
+  }
+}
+
+// Source pointers (at the thread's chunk, k-block 0) and shared-memory byte
+// offsets within a stage's A tile for the slots above; returns how many of
+// the thread's rows are inside the tile.  A slot outside [0, gather_T *
+// gather_k) is flagged and read as token 0 (the row's output is then
+// meaningless but every load stays in bounds).  Rows past the tile are not
+// copied: their accumulator rows are never stored.
+__device__ __forceinline__ int gather_rows_of_thread(const Params& p, const int (&slot)[kGatherRowsPerThread], int gt,
+                                                     const char* (&src)[kGatherRowsPerThread],
+                                                     uint32_t (&dst_off)[kGatherRowsPerThread]) {
+  const int c = gt & 7, rr = gt >> 3;  // chunk, first row (0..15)
+  int n = 0;
+#pragma unroll
+  for (int j = 0; j < kGatherRowsPerThread; ++j) {
+    const int row = rr + 16 * j;
+    src[j] = nullptr;
+    dst_off[j] = (uint32_t)row * 128u + (uint32_t)((c ^ (row & 7)) << 4);
+    if (slot[j] != -1) {
+      int t = slot[j] / p.gather_k;
+      if (slot[j] < 0 || t >= p.gather_T) {
+        flag_error(kErrBadRow);
+        t = 0;
+      }
+      src[j] = reinterpret_cast<const char*>(p.gather_x) + ((size_t)t * p.K + (size_t)c * 8) * 2;
+      n = j + 1;
+    }
+  }
+  return n;
+}
+
+// The k-blocks of one tile: wait for the stage to be free, copy this thread's
+// rows of the k-block (16 zero bytes where the chunk lies past K), arrive on
+// the stage's full barrier.  Returns false if a wait gave up.
+template <typename EmptyBar, typename FullBar>
+__device__ __forceinline__ bool gather_tile(const Params& p, int num_kb, int nrows,
+                                            const char* const (&src)[kGatherRowsPerThread],
+                                            const uint32_t (&dst_off)[kGatherRowsPerThread], uint32_t sA_base,
+                                            uint32_t a_stage_bytes, int nstages, int& stage, uint32_t& phase,
+                                            EmptyBar empty_bar, FullBar full_bar, volatile int* abort_flag) {
+  const int c8 = (int)(threadIdx.x & 7) * 8;  // this thread's first K element within a k-block
+  for (int kb = 0; kb < num_kb; ++kb) {
+    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) return false;
+    const uint32_t base = sA_base + (uint32_t)stage * a_stage_bytes;
+    const uint32_t nbytes = kb * BK + c8 < p.K ? 16u : 0u;
+    const size_t koff = (size_t)kb * BK * 2;
+#pragma unroll
+    for (int j = 0; j < kGatherRowsPerThread; ++j)
+      if (j < nrows && src[j] != nullptr) cp_async16(base + dst_off[j], nbytes ? src[j] + koff : src[j], nbytes);
+    cp_async_arrive_noinc(full_bar(stage));
+    if (++stage == nstages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+  return true;
+}
 
 template <bool GATEUP, int BN, int STAGES>
 struct Cfg {
@@ -248,8 +362,8 @@ struct Cfg {
   static_assert(!GATEUP || BN % 64 == 0, "gate/up halves must be whole 64-column boxes");
 };
 
-template <bool GATEUP, int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool GATEUP, int BN, int STAGES, bool GATHER = false>
+__global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b0,
                            const __grid_constant__ CUtensorMap tmap_b1, Params p) {
   using C = Cfg<GATEUP, BN, STAGES>;
@@ -273,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), GATHER ? 1 + kGatherThreads : 1);  // + one cp.async arrival per gather thread
       mbar_init(empty_bar(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -284,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    prefetch_tmap(&tmap_a);
+    if (!GATHER) prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b0);
     if (GATEUP) prefetch_tmap(&tmap_b1);
   }
@@ -368,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (lane == 0) {  // (weights only when warps 6..9 gather the A rows)
       int stage = 0;
       uint32_t phase = 0, armed_mask = 0, armed_par = 0;
       bool ok = true;
@@ -383,12 +497,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, C::kStageBytes);
+          mbar_arrive_expect_tx(fb, GATHER ? C::kBBytes : C::kStageBytes);
           armed_mask |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           const uint32_t a_dst = smem_u32(sA + (size_t)stage * kABytes);
           const uint32_t b_dst = smem_u32(sB + (size_t)stage * C::kBBytes);
-          tma_load_2d_h<MOE_TC_HINT_A>(a_dst, &tmap_a, fb, kb * BK, m0, pol_a);
+          if (!GATHER) tma_load_2d_h<MOE_TC_HINT_A>(a_dst, &tmap_a, fb, kb * BK, m0, pol_a);
           if (GATEUP) {
             constexpr int HB = C::NBOX / 2;  // boxes per half
 #pragma unroll
@@ -441,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (GATHER && MOE_TC_GATHER_FENCE) fence_proxy_async_smem();  // the A rows came through cp.async
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + (size_t)stage * kABytes);
           const uint32_t b_addr = smem_u32(sB + (size_t)stage * C::kBBytes);
@@ -468,6 +583,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (GATHER && warp >= 6) {
+    // ------------------------------------------------ A-row gather (warps 6..9)
+    const int gt = (int)threadIdx.x - 192;
+    int stage = 0;
+    uint32_t phase = 0;
+    // rows of this CTA's part of a tile (an M=64 tile reads 64 rows)
+    auto tile_rows = [&](int tile, int& r0, int& r_end) {
+      int e, m0, mend, n0;
+      tile_coords(tile, e, m0, mend, n0);
+      r0 = m0;
+      r_end = min(mend, m0 + ((MOE_TC_M64 && (mend - m0 <= 64)) ? 64 : BM));
+    };
+    int slot[kGatherRowsPerThread];
+    int tile = blockIdx.x;
+    if (tile < total_tiles) {
+      int r0, r_end;
+      tile_rows(tile, r0, r_end);
+      gather_load_slots(p, r0, r_end, gt, slot);
+    }
+    for (; tile < total_tiles; tile += gridDim.x) {
+      const char* src[kGatherRowsPerThread];
+      uint32_t dst_off[kGatherRowsPerThread];
+      const int nrows = gather_rows_of_thread(p, slot, gt, src, dst_off);
+      if (tile + (int)gridDim.x < total_tiles) {  // next tile's slots, in flight during this one
+        int r0, r_end;
+        tile_rows(tile + (int)gridDim.x, r0, r_end);
+        gather_load_slots(p, r0, r_end, gt, slot);
+      }
+      if (!gather_tile(p, num_kb, nrows, src, dst_off, smem_u32(sA), kABytes, STAGES, stage, phase,
+                       [&](int s) { return empty_bar(s); }, [&](int s) { return full_bar(s); }, s_abort))
+        break;
+    }
+    cp_async_wait_all();
   } else {
     // ------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -602,11 +750,11 @@ inline int num_sms() {
   });
 }
 
-template <bool GATEUP, int BN, int STAGES>
+template <bool GATEUP, int BN, int STAGES, bool GATHER = false>
 cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const Params& p,
                       cudaStream_t stream) {
   using C = Cfg<GATEUP, BN, STAGES>;
-  auto kern = grouped_gemm_tc_kernel<GATEUP, BN, STAGES>;
+  auto kern = grouped_gemm_tc_kernel<GATEUP, BN, STAGES, GATHER>;
   const size_t smem = C::smem_bytes(p.E);
   static PerDeviceOnce attr_once;  // the attribute is per device; set it once for the largest E
   cudaError_t err = attr_once.run(current_device(), [&] {
@@ -616,7 +764,7 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUten
   const long long max_tiles = ((long long)(p.S + BM - 1) / BM + p.E) * p.ntn;
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
-  err = launch_pdl(kern, grid, kThreads, smem, stream, ta, tb0, tb1, p);
+  err = launch_pdl(kern, grid, GATHER ? kThreads + kGatherThreads : kThreads, smem, stream, ta, tb0, tb1, p);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
@@ -627,8 +775,20 @@ inline cudaError_t launch_gate_up(const void* x_disp, const void* wg, const void
   CUtensorMap ta, tg, tu;
   if (!make_tmap_act(&ta, x_disp, S, H) || !make_tmap_weight(&tg, wg, E, H, I) || !make_tmap_weight(&tu, wu, E, H, I))
     return cudaErrorInvalidValue;
-  Params p{off, E, S, H, I, (I + 127) / 128, reinterpret_cast<__nv_bfloat16*>(h)};
+  Params p{off, E, S, H, I, (I + 127) / 128, reinterpret_cast<__nv_bfloat16*>(h), nullptr, 1, 0, nullptr};
   return launch_tc<true, 128, 4>(ta, tg, tu, p, stream);
+}
+
+// launch_gate_up with the A rows gathered from x [T, H]: dispatched row r is
+// token row_to_slot[r] / k (x_disp is never formed).
+inline cudaError_t launch_gate_up_gather(const void* x, int T, const int32_t* row_to_slot, int k, const void* wg,
+                                         const void* wu, const int32_t* off, int E, int H, int I, int S, void* h,
+                                         cudaStream_t stream) {
+  if (S == 0) return cudaSuccess;
+  CUtensorMap tg, tu;  // the A rows come from x through cp.async: no activation tensor map
+  if (!make_tmap_weight(&tg, wg, E, H, I) || !make_tmap_weight(&tu, wu, E, H, I)) return cudaErrorInvalidValue;
+  Params p{off, E, S, H, I, (I + 127) / 128, reinterpret_cast<__nv_bfloat16*>(h), row_to_slot, k, T, x};
+  return launch_tc<true, 128, 4, true>(tg, tg, tu, p, stream);
 }
 
 // y_disp = h Wd; n-tile width chosen to cover H with the least padding
@@ -652,7 +812,7 @@ inline cudaError_t launch_down(const void* h, const void* wd, const int32_t* off
     }
   }
   if (MOE_TC_DOWN_BN > 0) best = MOE_TC_DOWN_BN;
-  Params p{off, E, S, I, H, (H + best - 1) / best, reinterpret_cast<__nv_bfloat16*>(y)};
+  Params p{off, E, S, I, H, (H + best - 1) / best, reinterpret_cast<__nv_bfloat16*>(y), nullptr, 1, 0, nullptr};
   switch (best) {
     case 256:
       return launch_tc<false, 256, 4>(ta, tb, tb, p, stream);

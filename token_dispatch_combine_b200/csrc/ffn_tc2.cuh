@@ -14,6 +14,10 @@
 //     TMEM and arrives on the leader's "accumulator empty" barrier.
 // An expert's last tile, when at most 128 rows are left, is an M=128 pair MMA
 // (64 rows per CTA).
+// Gathering form: each CTA's gather threads copy its own A rows from x
+// (cp.async) and arrive on its own full barrier; in the peer an otherwise idle
+// thread (warp 1) waits for that barrier and arrives on the leader's, which
+// the MMA thread waits on.
 // Per CTA a stage is 16 KB of A + 16 KB of B, so the ring holds 6 stages
 // (half the weight bytes per SM of the single-CTA kernel, 50% more time of
 // work in flight).  No TMA multicast: every load brings one CTA's own data.
@@ -30,6 +34,14 @@ constexpr int BM2 = 256;  // rows of a pair tile (128 per CTA)
 // Pair m-tiles per raster group (tiles of a group share weight columns in L2).
 #ifndef MOE_TC2_GROUP_M
 #define MOE_TC2_GROUP_M 8
+#endif
+
+// Gathering pair kernel: semantics of the peer relay's arrival on the
+// leader's barrier: 0 release at CTA scope (mbarrier.arrive's default),
+// 1 relaxed, 2 release at cluster scope (measured: 2.4x slower kernel, the
+// cluster-scope release waits for the peer's copies still in flight).
+#ifndef MOE_TC2_RELAY
+#define MOE_TC2_RELAY 0
 #endif
 
 // An expert's last tile with at most 128 rows left runs as an M=128 pair MMA
@@ -57,6 +69,14 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Arrive on a barrier of another CTA of the cluster with release ordering at
+// CTA scope only (the default semantics of mbarrier.arrive), or none.
+__device__ __forceinline__ void mbar_arrive_remote_cta_release(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // TMA into this CTA's shared memory, completion counted on an mbarrier that may
 // live in the peer CTA (cta_group::2; not a multicast load).
@@ -115,8 +135,8 @@ struct Cfg2 {
   }
 };
 
-template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool GATEUP, bool GATHER = false>
+__global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_a64,
                             const __grid_constant__ CUtensorMap tmap_b0, const __grid_constant__ CUtensorMap tmap_b1,
                             Params p) {
@@ -144,7 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);   // leader's copy: its own arrive_expect_tx (bytes of both CTAs)
+      // leader's copy: its own arrive_expect_tx (bytes of both CTAs); when gathering
+      // also its gather threads' cp.async arrivals and the peer's relay.  The
+      // peer's copy (gathering only) counts the peer's gather threads.
+      mbar_init(full_bar(s), GATHER ? (rank == 0 ? 2 + kGatherThreads : kGatherThreads) : 1);
       mbar_init(empty_bar(s), 1);  // the leader's MMA commit, multicast to both CTAs
     }
     for (int a = 0; a < 2; ++a) {
@@ -155,8 +178,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    prefetch_tmap(&tmap_a);
-    if (MOE_TC2_HALF) prefetch_tmap(&tmap_a64);
+    if (!GATHER) {
+      prefetch_tmap(&tmap_a);
+      if (MOE_TC2_HALF) prefetch_tmap(&tmap_a64);
+    }
     prefetch_tmap(&tmap_b0);
     if (GATEUP) prefetch_tmap(&tmap_b1);
   }
@@ -234,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
+    if (lane == 0) {  // (weights only when warps 6..9 gather the A rows)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -247,13 +272,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          // a half tile brings 64 rows of A per CTA
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * (C::kStageBytes - (half ? kABytes / 2 : 0u)));
+          // a half tile brings 64 rows of A per CTA; gathered A rows are not TMA bytes
+          if (rank == 0)
+            mbar_arrive_expect_tx(full_bar(stage),
+                                  GATHER ? 2 * C::kBBytes : 2 * (C::kStageBytes - (half ? kABytes / 2 : 0u)));
           const uint32_t fb = mapa_shared(full_bar(stage), 0);  // the leader's full barrier
           const uint32_t a_dst = smem_u32(sA + (size_t)stage * kABytes);
           const uint32_t b_dst = smem_u32(sB + (size_t)stage * C::kBBytes);
-          if (half) tma_load_2d_pair(a_dst, &tmap_a64, fb, kb * BK, m0 + 64 * (int)rank);
-          else tma_load_2d_pair(a_dst, &tmap_a, fb, kb * BK, m0 + 128 * (int)rank);
+          if (!GATHER) {
+            if (half) tma_load_2d_pair(a_dst, &tmap_a64, fb, kb * BK, m0 + 64 * (int)rank);
+            else tma_load_2d_pair(a_dst, &tmap_a, fb, kb * BK, m0 + 128 * (int)rank);
+          }
           if (GATEUP) {  // each CTA: [gate 64 | up 64] for h columns n0 + 64 * rank + [0, 64)
             const int c0 = n0 + 64 * (int)rank;
             tma_load_3d_pair(b_dst, &tmap_b0, fb, c0, kb * BK, e);
@@ -317,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (GATHER && MOE_TC_GATHER_FENCE) fence_proxy_async_smem();  // this CTA's A rows came through cp.async
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + (size_t)stage * kABytes);
           const uint32_t b_addr = smem_u32(sB + (size_t)stage * C::kBBytes);
@@ -339,8 +369,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit_pair(drain_bar, 0x1);
         mbar_wait(drain_bar, 0, nullptr, 100000000ull);
       }
+    } else if (GATHER && lane == 0 && rank == 1) {
+      // ---------------------------------------------- relay (peer, gathering only):
+      // once this CTA's gathered rows of a stage have landed, make them visible
+      // to the async proxy and tell the leader's full barrier.
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total_tiles; tile += ncl) {
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, s_abort)) {
+            ok = false;
+            break;
+          }
+          if (MOE_TC_GATHER_FENCE) fence_proxy_async_smem();
+          const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+          if (MOE_TC2_RELAY == 0) mbar_arrive_remote_cta_release(leader_full);
+          else if (MOE_TC2_RELAY == 1) mbar_arrive_cluster_relaxed(leader_full);
+          else mbar_arrive_cluster(leader_full);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
     }
     __syncwarp();
+  } else if (GATHER && warp >= 6) {
+    // ------------------------------------------------ A-row gather (warps 6..9, both CTAs):
+    // this CTA's rows of the pair tile, arrivals on this CTA's full barrier
+    const int gt = (int)threadIdx.x - 192;
+    int stage = 0;
+    uint32_t phase = 0;
+    auto tile_rows = [&](int tile, int& r0, int& r_end) {
+      int e, m0, mend, n0;
+      tile_coords(tile, e, m0, mend, n0);
+      const int arows = (MOE_TC2_HALF && (mend - m0 <= 128)) ? 64 : 128;  // rows of A per CTA
+      r0 = m0 + arows * (int)rank;
+      r_end = min(mend, r0 + arows);
+    };
+    int slot[kGatherRowsPerThread];
+    int tile = cid;
+    if (tile < total_tiles) {
+      int r0, r_end;
+      tile_rows(tile, r0, r_end);
+      gather_load_slots(p, r0, r_end, gt, slot);
+    }
+    for (; tile < total_tiles; tile += ncl) {
+      const char* src[kGatherRowsPerThread];
+      uint32_t dst_off[kGatherRowsPerThread];
+      const int nrows = gather_rows_of_thread(p, slot, gt, src, dst_off);
+      if (tile + ncl < total_tiles) {  // next tile's slots, in flight during this one
+        int r0, r_end;
+        tile_rows(tile + ncl, r0, r_end);
+        gather_load_slots(p, r0, r_end, gt, slot);
+      }
+      if (!gather_tile(p, num_kb, nrows, src, dst_off, smem_u32(sA), kABytes, STAGES, stage, phase,
+                       [&](int s) { return empty_bar(s); }, [&](int s) { return full_bar(s); }, s_abort))
+        break;
+    }
+    cp_async_wait_all();
   } else {
     // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -438,13 +526,13 @@ inline bool make_tmap_act64(CUtensorMap* m, const void* base, int rows, int K) {
 
 // Number of 2-CTA clusters that can be resident at once (each CTA takes one
 // SM), cached per device.
-template <bool GATEUP>
+template <bool GATEUP, bool GATHER>
 int max_pair_clusters(size_t smem) {
   static PerDeviceInt cached;
   return cached.get(current_device(), [&] {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms() / 2));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(GATHER ? kThreads + kGatherThreads : kThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -454,17 +542,17 @@ int max_pair_clusters(size_t smem) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tc2_kernel<GATEUP>, &cfg) != cudaSuccess || n <= 0)
+    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tc2_kernel<GATEUP, GATHER>, &cfg) != cudaSuccess || n <= 0)
       n = num_sms() / 2;
     return n;
   });
 }
 
-template <bool GATEUP>
+template <bool GATEUP, bool GATHER = false>
 cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& ta64, const CUtensorMap& tb0, const CUtensorMap& tb1,
                        const Params& p, cudaStream_t stream) {
   using C = Cfg2<GATEUP>;
-  auto kern = grouped_gemm_tc2_kernel<GATEUP>;
+  auto kern = grouped_gemm_tc2_kernel<GATEUP, GATHER>;
   const size_t smem = C::smem_bytes(p.E);
   static PerDeviceOnce attr_once;  // the attribute is per device; set it once for the largest E
   cudaError_t err = attr_once.run(current_device(), [&] {
@@ -472,11 +560,11 @@ cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& ta64, const CUt
   });
   if (err != cudaSuccess) return err;
   const long long max_tiles = ((long long)(p.S + BM2 - 1) / BM2 + p.E) * p.ntn;
-  long long clusters = max_pair_clusters<GATEUP>(C::smem_bytes(1024));
+  long long clusters = max_pair_clusters<GATEUP, GATHER>(C::smem_bytes(1024));
   if (max_tiles < clusters) clusters = max_tiles > 0 ? max_tiles : 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * clusters));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(GATHER ? kThreads + kGatherThreads : kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -500,8 +588,19 @@ inline cudaError_t launch_gate_up_pair(const void* x_disp, const void* wg, const
   if (!make_tmap_act(&ta, x_disp, S, H) || !make_tmap_act64(&ta64, x_disp, S, H) ||
       !make_tmap_weight(&tg, wg, E, H, I) || !make_tmap_weight(&tu, wu, E, H, I))
     return cudaErrorInvalidValue;
-  Params p{off, E, S, H, I, (I + 127) / 128, reinterpret_cast<__nv_bfloat16*>(h)};
+  Params p{off, E, S, H, I, (I + 127) / 128, reinterpret_cast<__nv_bfloat16*>(h), nullptr, 1, 0, nullptr};
   return launch_tc2<true>(ta, ta64, tg, tu, p, stream);
+}
+
+// launch_gate_up_pair with the A rows gathered from x [T, H] (see launch_gate_up_gather).
+inline cudaError_t launch_gate_up_pair_gather(const void* x, int T, const int32_t* row_to_slot, int k, const void* wg,
+                                              const void* wu, const int32_t* off, int E, int H, int I, int S, void* h,
+                                              cudaStream_t stream) {
+  if (S == 0) return cudaSuccess;
+  CUtensorMap tg, tu;  // the A rows come from x through cp.async: no activation tensor map
+  if (!make_tmap_weight(&tg, wg, E, H, I) || !make_tmap_weight(&tu, wu, E, H, I)) return cudaErrorInvalidValue;
+  Params p{off, E, S, H, I, (I + 127) / 128, reinterpret_cast<__nv_bfloat16*>(h), row_to_slot, k, T, x};
+  return launch_tc2<true, true>(tg, tg, tg, tu, p, stream);
 }
 
 inline cudaError_t launch_down_pair(const void* h, const void* wd, const int32_t* off, int E, int H, int I, int S,
@@ -510,7 +609,7 @@ inline cudaError_t launch_down_pair(const void* h, const void* wd, const int32_t
   CUtensorMap ta, ta64, tb;
   if (!make_tmap_act(&ta, h, S, I) || !make_tmap_act64(&ta64, h, S, I) || !make_tmap_weight(&tb, wd, E, I, H))
     return cudaErrorInvalidValue;
-  Params p{off, E, S, I, H, (H + 255) / 256, reinterpret_cast<__nv_bfloat16*>(y)};
+  Params p{off, E, S, I, H, (H + 255) / 256, reinterpret_cast<__nv_bfloat16*>(y), nullptr, 1, 0, nullptr};
   return launch_tc2<false>(ta, ta64, tb, tb, p, stream);
 }
 

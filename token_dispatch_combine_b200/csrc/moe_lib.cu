@@ -24,12 +24,19 @@ std::atomic<int> g_ffn_tiling{MOE_FFN_TILING_AUTO};
 // Pair tiles pad each expert's rows to 256 instead of 128; they pay off once
 // the average expert holds enough rows (measured: 512 rows per expert gain,
 // 256 lose).
-constexpr int kPairMinRowsPerExpert = 384;
+// Auto tiling: pair tiles from this many rows per expert on.  An expert whose
+// rows leave a remainder of at most 128 past a multiple of 256 ends in an
+// M=128 pair tile that costs about as much as a full one, so the gate/up
+// projection (the longer one) needs a few more rows per expert than down
+// before the pair tiles' lower per-row cost wins.
+constexpr int kPairMinRowsGateUp = 448;
+constexpr int kPairMinRowsDown = 384;
 
-int resolve_tiling(int E, int S) {
+int resolve_tiling(int E, int S, bool gate_up) {
   const int mode = g_ffn_tiling.load(std::memory_order_relaxed);
   if (mode != MOE_FFN_TILING_AUTO) return mode;
-  return (long long)S >= (long long)kPairMinRowsPerExpert * E ? MOE_FFN_TILING_PAIR : MOE_FFN_TILING_SINGLE;
+  const long long need = (long long)(gate_up ? kPairMinRowsGateUp : kPairMinRowsDown) * E;
+  return (long long)S >= need ? MOE_FFN_TILING_PAIR : MOE_FFN_TILING_SINGLE;
 }
 
 thread_local std::string g_last_msg;
@@ -69,7 +76,7 @@ moe_status check_k_e(int k, int E) {
 
 extern "C" {
 
-int moe_abi_version(void) { return 1; }
+int moe_abi_version(void) { return 2; }
 
 moe_status moe_set_ffn_tiling(int mode) {
   if (mode != MOE_FFN_TILING_AUTO && mode != MOE_FFN_TILING_SINGLE && mode != MOE_FFN_TILING_PAIR)
@@ -80,7 +87,10 @@ moe_status moe_set_ffn_tiling(int mode) {
 
 int moe_get_ffn_tiling(void) { return g_ffn_tiling.load(std::memory_order_relaxed); }
 
-int moe_ffn_tiling_for(int E, int S) { return E > 0 && S >= 0 ? resolve_tiling(E, S) : -1; }
+int moe_ffn_tiling_for(int E, int S, int projection) {
+  if (E <= 0 || S < 0 || (projection != MOE_FFN_GATE_UP && projection != MOE_FFN_DOWN)) return -1;
+  return resolve_tiling(E, S, projection == MOE_FFN_GATE_UP);
+}
 
 const char* moe_status_string(int status) {
   switch (status) {
@@ -157,10 +167,14 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
   MOE_REQUIRE_PTR(workspace, 16, "workspace");
   const moe::DispatchGeom g = moe::make_dispatch_geom(T, k, E, R);
   MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(g), "workspace_bytes smaller than moe_dispatch_workspace_bytes()");
+  MOE_REQUIRE((x == nullptr) == (x_disp == nullptr),
+              "x and x_disp must both be given, or both be NULL (index-only dispatch)");
   if (T > 0) {
-    MOE_REQUIRE_PTR(x, 16, "x");
+    if (x != nullptr) {
+      MOE_REQUIRE_PTR(x, 16, "x");
+      MOE_REQUIRE_PTR(x_disp, 16, "x_disp");
+    }
     MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
-    MOE_REQUIRE_PTR(x_disp, 16, "x_disp");
     MOE_REQUIRE_PTR(slot_to_row, 4, "slot_to_row");
     MOE_REQUIRE_PTR(row_to_slot, 4, "row_to_slot");
   }
@@ -261,7 +275,7 @@ moe_status moe_ffn_gate_up(const void* x_disp, int dtype, const void* w_gate, co
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t err;
   if (dtype == MOE_BF16)
-    err = resolve_tiling(E, S) == MOE_FFN_TILING_PAIR
+    err = resolve_tiling(E, S, true) == MOE_FFN_TILING_PAIR
               ? moe::tc::launch_gate_up_pair(x_disp, w_gate, w_up, expert_offsets, E, H, I, S, h, s)
               : moe::tc::launch_gate_up(x_disp, w_gate, w_up, expert_offsets, E, H, I, S, h, s);
   else
@@ -280,7 +294,7 @@ moe_status moe_ffn_down(const void* h, int dtype, const void* w_down, const int3
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t err;
   if (dtype == MOE_BF16)
-    err = resolve_tiling(E, S) == MOE_FFN_TILING_PAIR
+    err = resolve_tiling(E, S, false) == MOE_FFN_TILING_PAIR
               ? moe::tc::launch_down_pair(h, w_down, expert_offsets, E, H, I, S, y_disp, s)
               : moe::tc::launch_down(h, w_down, expert_offsets, E, H, I, S, y_disp, s);
   else
@@ -293,6 +307,43 @@ moe_status moe_expert_ffn(const void* x_disp, int dtype, const void* w_gate, con
                           const void* w_down, const int32_t* expert_offsets, int E, int H, int I, int S, void* h,
                           void* y_disp, void* stream) {
   moe_status st = moe_ffn_gate_up(x_disp, dtype, w_gate, w_up, expert_offsets, E, H, I, S, h, stream);
+  if (st != MOE_OK) return st;
+  return moe_ffn_down(h, dtype, w_down, expert_offsets, E, H, I, S, y_disp, stream);
+}
+
+moe_status moe_ffn_gate_up_gather(const void* x, int dtype, int T, const int32_t* row_to_slot, int k,
+                                  const void* w_gate, const void* w_up, const int32_t* expert_offsets, int E, int H,
+                                  int I, int S, void* h, void* stream) {
+  moe_status st = check_ffn(dtype, E, H, I, S, x, "x", expert_offsets);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  MOE_REQUIRE(k >= 1 && k <= 8, "k must be in [1, 8]");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  MOE_REQUIRE(S <= T * k, "S must be <= T * k");
+  if (S == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(row_to_slot, 4, "row_to_slot");
+  MOE_REQUIRE_PTR(w_gate, 16, "w_gate");
+  MOE_REQUIRE_PTR(w_up, 16, "w_up");
+  MOE_REQUIRE_PTR(h, 16, "h");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = resolve_tiling(E, S, true) == MOE_FFN_TILING_PAIR
+              ? moe::tc::launch_gate_up_pair_gather(x, T, row_to_slot, k, w_gate, w_up, expert_offsets, E, H, I, S,
+                                                    h, s)
+              : moe::tc::launch_gate_up_gather(x, T, row_to_slot, k, w_gate, w_up, expert_offsets, E, H, I, S, h, s);
+  else
+    err = moe::launch_ffn_simt_gate_up_gather((const float*)x, T, row_to_slot, k, (const float*)w_gate,
+                                              (const float*)w_up, expert_offsets, E, H, I, S, (float*)h, s);
+  return cuda_status(err, "moe_ffn_gate_up_gather");
+}
+
+moe_status moe_expert_ffn_gather(const void* x, int dtype, int T, const int32_t* row_to_slot, int k,
+                                 const void* w_gate, const void* w_up, const void* w_down,
+                                 const int32_t* expert_offsets, int E, int H, int I, int S, void* h, void* y_disp,
+                                 void* stream) {
+  moe_status st =
+      moe_ffn_gate_up_gather(x, dtype, T, row_to_slot, k, w_gate, w_up, expert_offsets, E, H, I, S, h, stream);
   if (st != MOE_OK) return st;
   return moe_ffn_down(h, dtype, w_down, expert_offsets, E, H, I, S, y_disp, stream);
 }
