@@ -53,17 +53,17 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def dram_traffic(workload: str):
-    """Per-launch DRAM bytes of the gate/up kernel from the committed ncu summary,
-    if it was taken on the current kernel source (else None)."""
+def dram_traffic(workload: str, gather: bool = False):
+    """Per-launch DRAM bytes of the gate/up kernel (its gathering form when `gather`)
+    from the committed ncu summary, if taken on the current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
     sha = kernel_source_sha()
     for line in open(path):
         parts = line.split()
-        if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload and parts[1] == "gate_up" \
-                and parts[3] == sha:
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload \
+                and parts[1] == ("gate_up_gather" if gather else "gate_up") and parts[3] == sha:
             return int(float(parts[2]))
     return None
 
@@ -172,6 +172,32 @@ def algorithmic(wl):
         "gateup_flops": 4.0 * S * wl.H * wl.I,
         "down_flops": 2.0 * S * wl.H * wl.I,
     }
+
+
+def gemm_bounds(wl, counts, gather, peaks):
+    """Roofline of the two grouped GEMMs from the layer's expert counts.
+
+    Per projection: algorithmic FLOPs and bytes (weights of the experts that have rows, the A rows
+    read once -- x itself when the gate/up projection gathers, the k-fold re-reads being L2 hits --
+    and the output written once), which of the two bounds the launch (time at the measured peak),
+    and the per-expert bound sum_e max(F_e / P_F, B_e / P_B) (each expert's weights stream while its
+    rows' products run)."""
+    b = 2 if wl.dtype == "bf16" else 4
+    H, I, S, T = wl.H, wl.I, wl.S, wl.T
+    P_F, P_B = peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9
+    counts = np.asarray(counts, np.float64)
+    active = counts > 0
+    out = {}
+    for proj, (w_elems, n_out, k_in, fl_per_row) in {
+            "gate_up": (2 * H * I, I, H, 4.0 * H * I), "down": (I * H, H, I, 2.0 * H * I)}.items():
+        flops = fl_per_row * S
+        a_rows = (T if (gather and proj == "gate_up") else S) * k_in * b
+        nbytes = active.sum() * w_elems * b + a_rows + S * n_out * b
+        f_e = fl_per_row * counts
+        b_e = active * w_elems * b + counts * (k_in + n_out) * b
+        out[proj] = {"flops": flops, "bytes": float(nbytes), "t_tensor": flops / P_F, "t_hbm": nbytes / P_B,
+                     "t_per_expert": float(np.maximum(f_e / P_F, b_e / P_B).sum())}
+    return out
 
 
 # --------------------------------------------------------------------------- CPU oracle legs
@@ -292,6 +318,7 @@ def run_ours(args, wl):
     st, bits = moe_get_error()
     if st != 0:
         raise RuntimeError(f"device error word {bits} during warm-up")
+    expert_counts = rt.disp.expert_counts.cpu().numpy()  # outside the timed region
 
     # Timed region: K whole steps, one event pair per step (no events between stages).
     def whole_step(a, b):
@@ -446,6 +473,19 @@ def run_ours(args, wl):
     peak_tf = peaks["bf16_tflops"]
     tiling = moe_ffn_tiling_for(wl.E, wl.S, FFN_GATE_UP)
     tiling_down = moe_ffn_tiling_for(wl.E, wl.S, FFN_DOWN)
+    bounds = gemm_bounds(wl, expert_counts, gather, peaks)
+    gu = bounds["gate_up"]
+    t_gu_s = t_gu * 1e-3
+    if gu["t_hbm"] > gu["t_tensor"]:  # the gate/up launch streams more bytes than its FLOPs need time
+        roof_bound, roof_unit, roof_peak = "hbm", "GB/s", peaks["hbm_gbs"]
+        roof_achieved = gu["bytes"] / t_gu_s / 1e9
+        roof_alg = (f"active gate+up weights + A rows + h = {gu['bytes']:.4g} B "
+                    f"(4*S*H*I = {gu['flops']:.4g} FLOP would take {gu['t_tensor'] * 1e6:.0f} us at peak)")
+    else:
+        roof_bound, roof_unit, roof_peak = "tensor", "TFLOP/s", peak_tf
+        roof_achieved = gu_tflops
+        roof_alg = f"4*S*H*I = {alg['gateup_flops']:.4g} FLOP"
+    gemm_bound_us = (bounds["gate_up"]["t_per_expert"] + bounds["down"]["t_per_expert"]) * 1e6
     cpu = None
     if args.cpu_baseline and world == 1:
         rng = np.random.default_rng(1)
@@ -480,6 +520,10 @@ def run_ours(args, wl):
             "stage_timing": "per-stage CUDA events in a separate pass of the same steps (each stage boundary "
                             "adds event overhead); back_to_back: one event pair around dispatch+combine; stream: 20 dispatch+combine pairs over 4 buffer sets (>L2) under one event pair",
             "grouped_gemm_tflops": gemm_tflops, "grouped_gemm_frac_bf16": gemm_tflops / peak_tf,
+            "grouped_gemm_bound_us": gemm_bound_us,
+            "grouped_gemm_frac_of_bound": gemm_bound_us / ((t_gu + t_down) * 1e3),
+            "grouped_gemm_bound": "sum over experts of max(FLOPs / bf16 peak, bytes / HBM peak), both "
+                                  "projections, from this layer's expert counts",
             **({} if router_ms is None else {
                 "router_topk_us": router_ms * 1e3,
                 "router_topk_gbs": alg["router_bytes"] / (router_ms * 1e-3) / 1e9,
@@ -495,10 +539,10 @@ def run_ours(args, wl):
                        if tiling == FFN_TILING_PAIR else
                        "grouped_gemm_tc_kernel<gate/up, SwiGLU epilogue" + (", rows gathered from x" if gather else "")
                        + "> (128-row tiles)"),
-            "bound": "tensor", "achieved": gu_tflops, "peak": peak_tf, "unit": "TFLOP/s",
-            "frac": gu_tflops / peak_tf, "traffic": dram_traffic(wl.name),
-            "peak_source": f"{peak_src} bf16 dense (burst)",
-            "algorithmic_per_launch": f"4*S*H*I = {alg['gateup_flops']:.4g} FLOP",
+            "bound": roof_bound, "achieved": roof_achieved, "peak": roof_peak, "unit": roof_unit,
+            "frac": roof_achieved / roof_peak, "traffic": dram_traffic(wl.name, gather),
+            "peak_source": f"{peak_src} " + ("bf16 dense (burst)" if roof_bound == "tensor" else "HBM copy"),
+            "algorithmic_per_launch": roof_alg,
         },
         "e2e": {"value": wl.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_np.nbytes + logits_np.nbytes), "d2h_bytes_per_step": int(y_h.numel() * y_h.element_size()),
