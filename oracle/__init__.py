@@ -50,6 +50,9 @@ def _configure(lib):
     lib.oracle_combine.argtypes = [vp, vp, vp, i32, i32, i32, vp]
     lib.oracle_router_logits.argtypes = [vp, i32, vp, i32, vp, i32, i32, i32, vp]
     lib.oracle_router_logits.restype = i32
+    lib.oracle_eplb_plan.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    lib.oracle_eplb_plan.restype = i32
+    lib.oracle_eplb_remap.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     return lib
 
 
@@ -223,3 +226,35 @@ def round_trip(x: np.ndarray, logits: np.ndarray, k: int, E: int, R: int, w_gate
         y_disp = np.concatenate([y_disp, np.zeros((S - n, H))])
     y = combine(y_disp, w, idx["slot_to_row"])
     return dict(ids=ids, w=w, x_disp=x_disp, act=act, y_disp=y_disp, y=y, **idx)
+
+
+def eplb_plan(load, R: int, slots: int) -> dict:
+    """Expert placement with replicas from per-expert loads (oracle_eplb_plan):
+    phys_to_logical [R*slots], replica_offsets [E+1], replicas [R*slots], and
+    the per-rank sum of replica shares the plan expects (rank_load [R])."""
+    load = _c(np.asarray(load), np.int64)
+    E = load.shape[0]
+    P = R * slots
+    p2l = np.full(P, -1, np.int32)
+    off = np.zeros(E + 1, np.int32)
+    reps = np.full(P, -1, np.int32)
+    st = _get().oracle_eplb_plan(load.ctypes.data, E, R, slots, p2l.ctypes.data, off.ctypes.data, reps.ctypes.data)
+    if st != 0:
+        raise ValueError("eplb_plan: need E, R, slots >= 1 and R * slots >= E")
+    n = np.diff(off)
+    rank_load = np.zeros(R, np.int64)
+    for e in range(E):
+        for j in range(n[e]):
+            share = load[e] // n[e] + (1 if j < load[e] % n[e] else 0)
+            rank_load[reps[off[e] + j] // slots] += share
+    return {"phys_to_logical": p2l, "replica_offsets": off, "replicas": reps, "rank_load": rank_load}
+
+
+def eplb_remap(ids: np.ndarray, E: int, replica_offsets: np.ndarray, replicas: np.ndarray) -> np.ndarray:
+    """Logical expert ids [T, k] -> physical replica ids (oracle_eplb_remap)."""
+    ids = _c(ids, np.int32)
+    T, k = ids.shape
+    out = np.empty_like(ids)
+    _get().oracle_eplb_remap(ids.ctypes.data, T, k, E, _c(replica_offsets, np.int32).ctypes.data,
+                             _c(replicas, np.int32).ctypes.data, out.ctypes.data)
+    return out

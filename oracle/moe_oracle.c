@@ -28,6 +28,10 @@
  *          sections "Weight Layout Across Ranks", "Collective Patterns /
  *          Prefill (CTE kernel)", "Why a Single All-Reduce/Reduce-Scatter
  *          Works", "Limitations" (items 1, 3 and 4).
+ *  [WIKI]  "什么是专家并行（Expert Parallelism）？" -- sections "工作机制"
+ *          (how it works) and "边界与常见误解" (third point): an expert-
+ *          parallel load balancer redistributes hot and cold experts over
+ *          the GPUs to keep their utilisation balanced.
  *  [SWIGLU] Shazeer, "GLU Variants Improve Transformer" (2020): FFN_SwiGLU(x)
  *          = (SiLU(x W) * (x V)) W2, SiLU(z) = z * sigmoid(z).  The pages call
  *          each expert "an MLP"; the layer shapes name its form SwiGLU.
@@ -255,4 +259,103 @@ void oracle_combine(const double* y_disp, const float* topk_w, const int32_t* sl
       for (int h = 0; h < H; ++h) out[h] += wj * y_disp[(size_t)row * H + h];
     }
   }
+}
+
+/* ----------------------------------------------------------------- EPLB
+ * [WIKI] "工作机制" / "边界与常见误解" (third point): routing is dynamic, so
+ * the per-expert token counts drift and a balancer redistributes hot and
+ * cold experts over the GPUs; [NEURON] "Limitations" 3: the static layout
+ * (rank r owns experts [r*E/R, (r+1)*E/R)) has no replication and no
+ * dynamic balancing.  The pages give no algorithm; this is the plainest
+ * reading, with every tie fixed so that results are exact integers:
+ *
+ *  plan (from measured per-expert loads, R ranks of `slots` physical expert
+ *  slots each, P = R * slots >= E):
+ *   1. every expert gets one replica; each of the P - E extra replicas goes
+ *      to the expert with the largest load per replica, load[e] / n[e]
+ *      (compared exactly as load[a] * n[b] vs load[b] * n[a]), ties to the
+ *      lower expert id;
+ *   2. replica j of expert e is given the share
+ *      load[e] / n[e] + (j < load[e] % n[e]) (integer division: an even
+ *      split of the expert's load);
+ *   3. replicas are placed one by one in order of decreasing share (ties:
+ *      lower expert id, then lower replica index), each on the rank with
+ *      the least placed share that still has a free slot (ties: lower
+ *      rank); it takes that rank's next slot, physical id rank*slots + i.
+ *  Outputs: phys_to_logical[P]; replica_offsets[E+1] (prefix sums of n) and
+ *  replicas[P] (physical ids of expert e's replicas j = 0..n[e]-1 at
+ *  replica_offsets[e] + j).  Returns -1 if P < E or a size is < 1.
+ *
+ *  remap (per step): slot t*k+j with logical expert e goes to replica
+ *  t mod n[e] of e (round robin over token indices); ids outside [0, E)
+ *  map to -1.
+ */
+int oracle_eplb_plan(const int64_t* load, int E, int R, int slots, int32_t* phys_to_logical,
+                     int32_t* replica_offsets, int32_t* replicas) {
+  if (E < 1 || R < 1 || slots < 1) return -1;
+  const int P = R * slots;
+  if (P < E) return -1;
+  int* n = (int*)malloc(sizeof(int) * (size_t)E);
+  for (int e = 0; e < E; ++e) n[e] = 1;
+  for (int extra = 0; extra < P - E; ++extra) {
+    int best = 0;
+    for (int e = 1; e < E; ++e)
+      if (load[e] * (int64_t)n[best] > load[best] * (int64_t)n[e]) best = e;
+    n[best] += 1;
+  }
+  replica_offsets[0] = 0;
+  for (int e = 0; e < E; ++e) replica_offsets[e + 1] = replica_offsets[e] + n[e];
+  /* the P replicas as (expert, index, share) */
+  int* item_e = (int*)malloc(sizeof(int) * (size_t)P);
+  int* item_j = (int*)malloc(sizeof(int) * (size_t)P);
+  int64_t* share = (int64_t*)malloc(sizeof(int64_t) * (size_t)P);
+  char* placed = (char*)calloc((size_t)P, 1);
+  int m = 0;
+  for (int e = 0; e < E; ++e)
+    for (int j = 0; j < n[e]; ++j) {
+      item_e[m] = e;
+      item_j[m] = j;
+      share[m] = load[e] / n[e] + (j < load[e] % n[e] ? 1 : 0);
+      ++m;
+    }
+  int64_t* rank_load = (int64_t*)calloc((size_t)R, sizeof(int64_t));
+  int* used = (int*)calloc((size_t)R, sizeof(int));
+  for (int step = 0; step < P; ++step) {
+    /* next: the unplaced item of largest share; items are listed by
+       (expert, index) ascending, so the first maximum wins ties */
+    int pick = -1;
+    for (int i = 0; i < P; ++i)
+      if (!placed[i] && (pick < 0 || share[i] > share[pick])) pick = i;
+    placed[pick] = 1;
+    int r_best = -1;
+    for (int r = 0; r < R; ++r)
+      if (used[r] < slots && (r_best < 0 || rank_load[r] < rank_load[r_best])) r_best = r;
+    const int phys = r_best * slots + used[r_best];
+    used[r_best] += 1;
+    rank_load[r_best] += share[pick];
+    phys_to_logical[phys] = item_e[pick];
+    replicas[replica_offsets[item_e[pick]] + item_j[pick]] = phys;
+  }
+  free(n);
+  free(item_e);
+  free(item_j);
+  free(share);
+  free(placed);
+  free(rank_load);
+  free(used);
+  return 0;
+}
+
+void oracle_eplb_remap(const int32_t* ids, int T, int k, int E, const int32_t* replica_offsets,
+                       const int32_t* replicas, int32_t* phys_ids) {
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[(size_t)t * k + j];
+      int out = -1;
+      if (e >= 0 && e < E) {
+        const int n = replica_offsets[e + 1] - replica_offsets[e];
+        out = replicas[replica_offsets[e] + t % n];
+      }
+      phys_ids[(size_t)t * k + j] = out;
+    }
 }

@@ -27,6 +27,8 @@ CASES = {
     "bf16_ragged": W("bf16_ragged", T=333, H=200, I=200, E=6, k=3, R=3, dtype="bf16", seed=12, bias="normal0.5"),
     "bf16_one_token": W("bf16_one_token", T=1, H=64, I=64, E=4, k=1, R=2, dtype="bf16", seed=14),
     "bf16_top8_e256": W("bf16_top8_e256", T=96, H=128, I=128, E=256, k=8, R=32, dtype="bf16", seed=16),
+    # the largest expert count: 1024-expert tile prefix in shared memory (gathered by default)
+    "bf16_e1024": W("bf16_e1024", T=2048, H=128, I=192, E=1024, k=8, R=8, dtype="bf16", seed=21),
     # ~512 rows per expert: full pair tiles, M=128 pair tails and single M=64 tails
     "bf16_pair_sized": W("bf16_pair_sized", T=2048, H=256, I=256, E=8, k=2, R=2, dtype="bf16", seed=22),
 }

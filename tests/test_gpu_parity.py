@@ -1,9 +1,9 @@
 """GPU round trip (through the C ABI) against the CPU oracle.
 
-These tests run the row-moving dispatch (x_disp is checked against the
-oracle's); the dispatch fused into the gate/up projection is checked in
-test_gpu_gather.py, and the host-pipeline and graph tests below run the
-round trip's default choice between the two.
+The small layers run the row-moving dispatch (x_disp is checked against the
+oracle's); the full-size layers, the host-pipeline and the graph tests run
+the round trip's default choice between that and the dispatch fused into
+the gate/up projection (checked on its own in test_gpu_gather.py).
 
 Integer outputs (ids, counts, offsets, permutation, dispatched rows) must be
 bit-exact; combination weights within 1e-6; float outputs within the
@@ -64,7 +64,8 @@ def check_routing_and_dispatch(layer: DeviceLayer, rt):
         got = dev_to_np(getattr(rt.disp, name))
         assert (got == ref[name]).all(), name
     x_disp = oracle.dispatch_rows(layer.x, wl.k, ref["slot_to_row"])
-    assert (dev_to_np(rt.disp.x_disp) == x_disp).all()
+    if rt.disp.x_disp is not None:  # (index-only dispatch when the gate/up projection gathers)
+        assert (dev_to_np(rt.disp.x_disp) == x_disp).all()
     return ids, w, ref, x_disp
 
 
@@ -109,9 +110,12 @@ def test_full_size_layer_other_tiling(name, ffn_tiling):
 
 
 def check_full_size_layer(name):
+    """The layer in the form bench.py times: MoERoundTrip's default dispatch (rows through x_disp,
+    or gathered by the gate/up projection where that is faster)."""
+    from token_dispatch_combine_b200 import MoERoundTrip
     wl = synth.WORKLOADS[name]
     layer = DeviceLayer(wl)
-    rt = run_gpu(layer)
+    rt = run_gpu(layer, MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, layer.x_dev.dtype))
     ids, w, ref, x_disp = check_routing_and_dispatch(layer, rt)
     rng = np.random.default_rng(wl.seed)
     S = wl.S

@@ -29,6 +29,13 @@ MUTANTS = {
     "combine_ignores_weight": ("out[h] += wj * y_disp", "out[h] += y_disp"),
     "router_weight_transposed": ("orc_load(w, wdt, (size_t)e * H + h)", "orc_load(w, wdt, (size_t)h * E + e)"),
     "router_drops_bias": ("      if (bias) acc += bias[e];\n", "\n"),
+    "eplb_extra_replica_to_lightest": ("if (load[e] * (int64_t)n[best] > load[best] * (int64_t)n[e]) best = e;",
+                                       "if (load[e] * (int64_t)n[best] < load[best] * (int64_t)n[e]) best = e;"),
+    "eplb_share_ignores_remainder": ("share[m] = load[e] / n[e] + (j < load[e] % n[e] ? 1 : 0);",
+                                     "share[m] = load[e] / n[e];"),
+    "eplb_places_on_heaviest_rank": ("(r_best < 0 || rank_load[r] < rank_load[r_best])",
+                                     "(r_best < 0 || rank_load[r] > rank_load[r_best])"),
+    "eplb_remap_first_replica_only": ("out = replicas[replica_offsets[e] + t % n];", "out = replicas[replica_offsets[e]];"),
     "combine_drops_last_choice": ("for (int j = 0; j < k; ++j) {\n      int row = slot_to_row", "for (int j = 0; j < k - 1; ++j) {\n      int row = slot_to_row"),
 }
 
@@ -48,6 +55,10 @@ PINS = [
     pins.test_router_logits_hand_example,
     pins.test_router_logits_one_hot_rows_select_columns,
     pins.test_router_logits_bias_only_and_bf16_widening,
+    pins.test_eplb_hand_example_one_hot_expert,
+    pins.test_eplb_equal_loads_without_extra_slots_alternate_ranks,
+    pins.test_eplb_remainders_go_to_the_first_replicas,
+    lambda: pins.test_eplb_plan_invariants(20, 4, 6, 3),
 ]
 
 

@@ -336,3 +336,75 @@ def test_router_then_route_reproduces_worked_example():
     ids, w = oracle.route(lg, g["k"])
     assert ids.tolist() == g["expected"]["topk_ids"]
     assert w.tolist() == g["expected"]["topk_w"]
+
+
+# ---------------------------------------------------------------- EPLB (expert placement with replicas)
+# "什么是专家并行（Expert Parallelism）？", 工作机制 / 边界与常见误解 (third point): a balancer
+# redistributes hot and cold experts over the GPUs.  The expected values below are worked by hand
+# from the reading stated in the oracle (greedy replica counts, even integer split of an expert's
+# load over its replicas, heaviest share first onto the least-loaded rank with a free slot).
+
+def test_eplb_hand_example_one_hot_expert():
+    # loads [8,1,...,1], 2 ranks x 5 slots: both extra replicas go to expert 0 (8/1, then 8/2 > 1);
+    # shares 3,3,2 then seven 1s; placement r0,r1,r0 (tie),r1,r1,r0 (tie),r1,r0 (tie),r1,r0 (r1 full)
+    p = oracle.eplb_plan([8, 1, 1, 1, 1, 1, 1, 1], 2, 5)
+    assert p["phys_to_logical"].tolist() == [0, 0, 3, 5, 7, 0, 1, 2, 4, 6]
+    assert p["replica_offsets"].tolist() == [0, 3, 4, 5, 6, 7, 8, 9, 10]
+    assert p["replicas"].tolist() == [0, 5, 1, 6, 7, 2, 8, 3, 9, 4]
+    assert p["rank_load"].tolist() == [8, 7]
+    # the static layout of the pages would put experts 0-3 on rank 0: loads 11 and 4
+    ids = np.array([[0], [0], [0], [1], [0], [9]], np.int32)
+    phys = oracle.eplb_remap(ids, 8, p["replica_offsets"], p["replicas"])
+    # token t goes to replica t mod 3 of expert 0 (phys 0, 5, 1), expert 1 has one replica, 9 is no expert
+    assert phys.ravel().tolist() == [0, 5, 1, 6, 5, -1]
+
+
+def test_eplb_equal_loads_without_extra_slots_alternate_ranks():
+    # 8 experts, 2 ranks x 4 slots, equal loads: no replicas; experts in id order alternate ranks
+    p = oracle.eplb_plan([5] * 8, 2, 4)
+    assert p["phys_to_logical"].tolist() == [0, 2, 4, 6, 1, 3, 5, 7]
+    assert p["replica_offsets"].tolist() == list(range(9))
+    assert p["rank_load"].tolist() == [20, 20]
+
+
+def test_eplb_remainders_go_to_the_first_replicas():
+    # one expert of load 7 over 3 slots on 1 rank: shares 3, 2, 2 (7 = 3 + 2 + 2)
+    p = oracle.eplb_plan([7], 1, 3)
+    assert p["replica_offsets"].tolist() == [0, 3]
+    assert p["replicas"].tolist() == [0, 1, 2]
+    assert p["rank_load"].tolist() == [7]
+    # two experts 10 and 4 on 2 ranks x 2 slots: extras to 10 (10/1 > 4, then 10/2 = 5 > 4);
+    # shares 4, 3, 3 (expert 0) and 4 (expert 1); order (0,0,4) -> r0 slot 0, (1,0,4) -> r1 slot 2,
+    # (0,1,3) -> r0 slot 1 (tie 4/4), (0,2,3) -> r1 slot 3
+    p = oracle.eplb_plan([10, 4], 2, 2)
+    assert p["replica_offsets"].tolist() == [0, 3, 4]
+    assert p["replicas"].tolist() == [0, 1, 3, 2]
+    assert p["phys_to_logical"].tolist() == [0, 0, 1, 0]
+    assert p["rank_load"].tolist() == [7, 7]
+
+
+@pytest.mark.parametrize("E,R,slots,seed", [(32, 8, 5, 1), (256, 32, 9, 2), (20, 4, 6, 3), (7, 3, 3, 4)])
+def test_eplb_plan_invariants(E, R, slots, seed):
+    rng = np.random.default_rng(seed)
+    load = (rng.zipf(1.3, E) * 17).astype(np.int64) % 5000
+    p = oracle.eplb_plan(load, R, slots)
+    P = R * slots
+    p2l, off, reps = p["phys_to_logical"], p["replica_offsets"], p["replicas"]
+    n = np.diff(off)
+    assert n.min() >= 1 and n.sum() == P and off[0] == 0
+    assert sorted(reps.tolist()) == list(range(P))             # every physical slot used once
+    for e in range(E):
+        assert (p2l[reps[off[e]:off[e + 1]]] == e).all()          # replicas point back to their expert
+    assert np.bincount(p2l, minlength=E).tolist() == n.tolist()
+    # greedy replica counts: no expert holding an extra replica would have less load per replica
+    # than another expert would with one more replica
+    for a in range(E):
+        if n[a] > 1:
+            for b in range(E):
+                assert load[a] * n[b] >= load[b] * (n[a] - 1)
+    # the expected rank loads add up to the total; the plan never loads a rank above the static
+    # layout's heaviest rank
+    assert p["rank_load"].sum() == load.sum()
+    static = load[: (E // R) * R].reshape(R, -1).sum(1).max() if E % R == 0 else None
+    if static is not None:
+        assert p["rank_load"].max() <= static
