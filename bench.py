@@ -430,6 +430,46 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         router_ms = sum(a.elapsed_time(b) for a, b in rev) / args.steps
         del w_router, r_ids, r_w
+    # Expert placement with replicas (one spare physical slot per logical rank), planned on the
+    # warm-up's expert counts: the busiest rank's rows before and after, the remap kernel's time,
+    # and the whole balanced step (route, remap, dispatch, FFN, combine over the replicas).
+    eplb = None
+    if wl.R > 1:
+        from token_dispatch_combine_b200 import MoEBalancedRoundTrip, moe_eplb_plan, moe_eplb_remap
+        slots = wl.E // wl.R + 1
+        plan = moe_eplb_plan(expert_counts, wl.R, slots, device=dev)
+        bal = MoEBalancedRoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, slots, dt, device=dev)
+        bal.set_plan(plan, wg, wu, wd)
+        for _ in range(3):
+            bal.forward(x, logits)
+        torch.cuda.synchronize()
+        before = rt.disp.rank_counts.cpu().numpy().astype(np.float64)
+        after = bal.rt.disp.rank_counts.cpu().numpy().astype(np.float64)
+        ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for (a, b), (c, d) in zip(ev_r, ev_s):
+            flush_and_hold()
+            a.record(stream)
+            moe_eplb_remap(bal.logical_ids, plan, out=bal.rt.topk_ids)
+            b.record(stream)
+            flush_and_hold()
+            c.record(stream)
+            bal.forward(x, logits)
+            d.record(stream)
+        torch.cuda.synchronize()
+        st, bits = moe_get_error()
+        if st != 0:
+            raise RuntimeError(f"device error word {bits} in the balanced round trip")
+        eplb = {
+            "physical_experts": plan.P, "slots_per_rank": slots,
+            "rank_rows_max_over_mean_static": float(before.max() / before.mean()),
+            "rank_rows_max_over_mean_balanced": float(after.max() / after.mean()),
+            "remap_us": statistics.median(a.elapsed_time(b) for a, b in ev_r) * 1e3,
+            "balanced_step_ms": statistics.median(c.elapsed_time(d) for c, d in ev_s),
+            "note": "plan from the warm-up's expert counts; a replica has its expert's weights, so outputs "
+                    "are unchanged; on one GPU the ranks are logical, so the step time shows the remap's cost",
+        }
+        del bal
     step_ms, dc_pair_ms, dc_stream_ms, t_disp_rows, t_comb_rows, *stage_max = max_over_ranks(
         [step_ms, dc_pair_ms, dc_stream_ms, *dc_stage, *stage.tolist()], world)
     if router_ms is not None:
@@ -530,6 +570,7 @@ def run_ours(args, wl):
                 "router_topk_frac_hbm": alg["router_bytes"] / (router_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "router_topk_timing": "moe_router_topk (logits = x W_r^T + bias, then top-k), L2 flushed, "
                                       "events per call; bytes T*H*2 + E*H*2 + T*k*8"}),
+            **({} if eplb is None else {"eplb": eplb}),
             "ffn_tiling": {"gate_up": "pair" if tiling == FFN_TILING_PAIR else "single",
                            "down": "pair" if tiling_down == FFN_TILING_PAIR else "single"},
         },

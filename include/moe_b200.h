@@ -279,6 +279,53 @@ moe_status moe_combine(const void* y_disp, int dtype, const float* topk_w, const
                        int H, void* y, void* stream);
 
 /*
+ * Expert placement with replicas -- an expert-parallel load balancer:
+ * "什么是专家并行（Expert Parallelism）？", "工作机制" and "边界与常见误解"
+ * (third point): routing is dynamic, so a balancer redistributes hot and cold
+ * experts over the GPUs to keep their utilisation balanced ("Expert
+ * Parallelism (EP)", "Limitations" 3: the static layout has neither).
+ *
+ * moe_eplb_plan (HOST arrays, runs on the CPU, no device work): from
+ * measured per-expert loads (e.g. expert_counts of earlier steps) place
+ * P = R * slots_per_rank physical experts, rank r holding physical ids
+ * [r * slots_per_rank, (r + 1) * slots_per_rank):
+ *   1. every expert gets one replica; each extra slot goes to the expert
+ *      with the largest load per replica (load[a] * n[b] vs load[b] * n[a]),
+ *      ties to the lower id;
+ *   2. replica j of expert e carries the share load[e] / n[e] +
+ *      (j < load[e] % n[e]);
+ *   3. largest share first (ties: lower expert, lower replica), each replica
+ *      takes the next slot of the rank with the least placed share that has
+ *      a free slot (ties: lower rank).
+ *   load            [E] int64, each in [0, 2^40)
+ *   phys_to_logical [P] int32 out: expert whose weights physical id p holds
+ *   replica_offsets [E + 1] int32 out: prefix sums of the replica counts
+ *   replicas        [P] int32 out: physical ids of expert e's replicas at
+ *                   replica_offsets[e] + j, j = 0 .. n_e - 1
+ * Needs E, R, slots_per_rank >= 1 and E <= P <= 2^20, else
+ * MOE_ERR_INVALID_ARG.  The result is an exact function of the inputs.
+ *
+ * moe_eplb_remap (device): phys_ids[t*k + j] = replicas[replica_offsets[e] +
+ * t mod n_e] for e = topk_ids[t*k + j] (a token's slots go round robin over
+ * the expert's replicas).  Ids outside [0, E) give -1 and set bit 1 of the
+ * error word; inconsistent replica tables give -1 and set bit 2.  Feed
+ * phys_ids to moe_dispatch with P experts and R ranks: the per-rank counts
+ * are then those of the plan.
+ *
+ * moe_eplb_replicate (device copies, phys_to_logical is a HOST array): the
+ * weights of the P physical experts, w_phys[p] = w[phys_to_logical[p]], each
+ * expert_bytes long (one cudaMemcpyAsync each).  A replica holds its
+ * expert's weights, so the round trip over the physical experts gives the
+ * same outputs, bit for bit, as the one over the logical experts.
+ */
+moe_status moe_eplb_plan(const int64_t* load, int E, int R, int slots_per_rank, int32_t* phys_to_logical,
+                         int32_t* replica_offsets, int32_t* replicas);
+moe_status moe_eplb_remap(const int32_t* topk_ids, int T, int k, int E, const int32_t* replica_offsets,
+                          const int32_t* replicas, int P, int32_t* phys_ids, void* stream);
+moe_status moe_eplb_replicate(const void* w, size_t expert_bytes, int E, const int32_t* phys_to_logical, int P,
+                              void* w_phys, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the current device's error word.
  * Returns MOE_OK, MOE_ERR_DEVICE (bad ids/offsets/rows were skipped),
  * MOE_ERR_TIMEOUT (a bounded wait ran out; outputs of that call are

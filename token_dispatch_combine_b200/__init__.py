@@ -7,7 +7,8 @@ the same names (``api``).  Importing it builds/loads the library and raises
 if that is impossible: there is no other implementation to fall back to.
 """
 from . import _native
-from .api import (DispatchOut, MoEHostPipeline, MoERoundTrip, moe_combine, moe_dispatch, moe_dispatch_workspace_bytes,
+from .api import (DispatchOut, EplbPlan, MoEBalancedRoundTrip, MoEHostPipeline, MoERoundTrip, moe_combine, moe_dispatch,
+                  moe_dispatch_workspace_bytes, moe_eplb_plan, moe_eplb_remap, moe_eplb_replicate,
                   moe_expert_ffn, moe_expert_ffn_gather, moe_ffn_down, moe_ffn_gate_up, moe_ffn_gate_up_gather,
                   moe_ffn_tiling_for, moe_get_error, moe_get_ffn_tiling, moe_route, moe_router_topk,
                   moe_set_ffn_tiling, new_dispatch_workspace)
@@ -20,5 +21,5 @@ __all__ = [
     "moe_expert_ffn", "moe_expert_ffn_gather", "moe_ffn_down", "moe_ffn_gate_up", "moe_ffn_gate_up_gather",
     "moe_get_error", "moe_route", "new_dispatch_workspace", "moe_set_ffn_tiling", "moe_get_ffn_tiling",
     "moe_ffn_tiling_for", "FFN_TILING_AUTO", "FFN_TILING_SINGLE", "FFN_TILING_PAIR", "FFN_GATE_UP", "FFN_DOWN",
-    "moe_router_topk",
+    "moe_router_topk", "EplbPlan", "MoEBalancedRoundTrip", "moe_eplb_plan", "moe_eplb_remap", "moe_eplb_replicate",
 ]

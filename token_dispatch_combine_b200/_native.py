@@ -24,7 +24,7 @@ EXPORTS = (
     "moe_abi_version", "moe_status_string", "moe_last_error_message", "moe_route", "moe_dispatch_workspace_bytes",
     "moe_dispatch", "moe_expert_ffn", "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_get_error", "moe_selftest_wait_timeout",
     "moe_dispatch_noalloc", "moe_set_ffn_tiling", "moe_get_ffn_tiling", "moe_ffn_tiling_for", "moe_router_topk",
-    "moe_ffn_gate_up_gather", "moe_expert_ffn_gather",
+    "moe_ffn_gate_up_gather", "moe_expert_ffn_gather", "moe_eplb_plan", "moe_eplb_remap", "moe_eplb_replicate",
 )
 
 _lock = threading.Lock()
@@ -59,6 +59,9 @@ def _configure(lib):
         "moe_ffn_tiling_for": ([i32, i32, i32], i32),
         "moe_ffn_gate_up_gather": ([vp, i32, i32, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp], i32),
         "moe_expert_ffn_gather": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp], i32),
+        "moe_eplb_plan": ([vp, i32, i32, i32, vp, vp, vp], i32),
+        "moe_eplb_remap": ([vp, i32, i32, i32, vp, vp, i32, vp, vp], i32),
+        "moe_eplb_replicate": ([vp, sz, i32, vp, i32, vp, vp], i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)

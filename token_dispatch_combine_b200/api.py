@@ -9,6 +9,7 @@ from __future__ import annotations
 import ctypes
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 from . import _native
@@ -309,6 +310,113 @@ class MoERoundTrip:
             self.forward(x, logits, w_gate, w_up, w_down, stream=s, y=y)
         torch.cuda.current_stream(self.device).wait_stream(s)
         return g
+
+
+@dataclass
+class EplbPlan:
+    """Placement of P = R * slots physical experts (replicas of the E logical ones)
+    from moe_eplb_plan; host arrays plus device copies of the remap tables."""
+    E: int
+    R: int
+    slots: int
+    phys_to_logical: np.ndarray   # [P] int32
+    replica_offsets: np.ndarray   # [E + 1] int32
+    replicas: np.ndarray          # [P] int32
+    replica_offsets_dev: torch.Tensor
+    replicas_dev: torch.Tensor
+
+    @property
+    def P(self) -> int:
+        return self.R * self.slots
+
+    def replica_counts(self) -> np.ndarray:
+        return np.diff(self.replica_offsets)
+
+
+def moe_eplb_plan(load, R: int, slots_per_rank: int, device="cuda") -> EplbPlan:
+    """Plan replicas and their placement on R ranks of slots_per_rank physical experts from
+    per-expert loads (numpy or torch, any integer dtype; e.g. expert_counts of earlier steps)."""
+    if isinstance(load, torch.Tensor):
+        load = load.detach().cpu().numpy()
+    load = np.ascontiguousarray(np.asarray(load, dtype=np.int64))
+    E = int(load.shape[0])
+    P = int(R) * int(slots_per_rank)
+    p2l = np.empty(max(P, 0), np.int32)
+    off = np.empty(E + 1, np.int32)
+    reps = np.empty(max(P, 0), np.int32)
+    check(_native.lib().moe_eplb_plan(load.ctypes.data, E, int(R), int(slots_per_rank), p2l.ctypes.data,
+                                      off.ctypes.data, reps.ctypes.data), "moe_eplb_plan")
+    return EplbPlan(E, int(R), int(slots_per_rank), p2l, off, reps,
+                    torch.from_numpy(off).to(device), torch.from_numpy(reps).to(device))
+
+
+def moe_eplb_remap(topk_ids: torch.Tensor, plan: EplbPlan, out: torch.Tensor | None = None, stream=None):
+    """Logical expert ids [T, k] -> physical replica ids (round robin over token index)."""
+    T, k = topk_ids.shape
+    if out is None:
+        out = torch.empty_like(topk_ids)
+    i32 = torch.int32
+    check(_native.lib().moe_eplb_remap(
+        _ptr(topk_ids, "topk_ids", i32), T, k, plan.E, _ptr(plan.replica_offsets_dev, "replica_offsets", i32),
+        _ptr(plan.replicas_dev, "replicas", i32), plan.P, _ptr(out, "phys_ids", i32), _stream(stream)),
+        "moe_eplb_remap")
+    return out
+
+
+def moe_eplb_replicate(w: torch.Tensor, plan: EplbPlan, out: torch.Tensor | None = None, stream=None):
+    """Weights of the physical experts: out[p] = w[plan.phys_to_logical[p]] (w is [E, ...])."""
+    if w.shape[0] != plan.E:
+        raise ValueError(f"w has {w.shape[0]} experts, the plan {plan.E}")
+    if out is None:
+        out = torch.empty((plan.P, *w.shape[1:]), dtype=w.dtype, device=w.device)
+    _ptr(w, "w")
+    _ptr(out, "out", w.dtype)
+    expert_bytes = w[0].numel() * w.element_size()
+    check(_native.lib().moe_eplb_replicate(w.data_ptr(), expert_bytes, plan.E, plan.phys_to_logical.ctypes.data,
+                                           plan.P, out.data_ptr(), _stream(stream)), "moe_eplb_replicate")
+    return out
+
+
+class MoEBalancedRoundTrip:
+    """The round trip over replicated experts: route on the E logical experts, remap each
+    slot to a physical replica (moe_eplb_remap), then dispatch, FFN and combine over the
+    P = R * slots_per_rank physical experts, rank r holding physical experts
+    [r * slots_per_rank, (r + 1) * slots_per_rank).  Outputs equal MoERoundTrip's bit for
+    bit (a replica has its expert's weights); the per-rank row counts follow the plan.
+    ``set_plan`` installs a plan and copies the weights of its physical experts."""
+
+    def __init__(self, T, H, I, E, k, R, slots_per_rank, dtype, device="cuda", gather="auto"):
+        self.E, self.k, self.R, self.slots = E, k, R, slots_per_rank
+        self.P = R * slots_per_rank
+        self.rt = MoERoundTrip(T, H, I, self.P, k, R, dtype, device=device, gather=gather)
+        self.logical_ids = torch.empty((T, k), dtype=torch.int32, device=self.rt.device)
+        self.plan = None
+        self.w = None
+
+    def set_plan(self, plan: EplbPlan, w_gate, w_up, w_down, stream=None):
+        if plan.E != self.E or plan.R != self.R or plan.slots != self.slots:
+            raise ValueError("plan sizes differ from the round trip's")
+        if self.w is None:
+            self.w = [torch.empty((self.P, *w.shape[1:]), dtype=w.dtype, device=w.device)
+                      for w in (w_gate, w_up, w_down)]
+        for dst, w in zip(self.w, (w_gate, w_up, w_down)):
+            moe_eplb_replicate(w, plan, out=dst, stream=stream)
+        self.plan = plan
+
+    def route(self, logits, stream=None):
+        moe_route(logits, self.k, self.logical_ids, self.rt.topk_w, stream)
+        return moe_eplb_remap(self.logical_ids, self.plan, out=self.rt.topk_ids, stream=stream)
+
+    def forward(self, x, logits, stream=None, y=None):
+        if self.plan is None:
+            raise RuntimeError("set_plan first")
+        self.route(logits, stream)
+        self.rt.dispatch(x, stream)
+        self.rt.gate_up(self.w[0], self.w[1], stream)
+        self.rt.down(self.w[2], stream)
+        return self.rt.combine(stream, y)
+
+    KERNELS_PER_FORWARD = 6  # route, remap, dispatch, gate/up, down, combine
 
 
 class MoEHostPipeline:

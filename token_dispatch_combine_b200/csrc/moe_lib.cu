@@ -15,6 +15,7 @@
 #include "ffn_tc.cuh"
 #include "ffn_tc2.cuh"
 #include "route.cuh"
+#include "eplb.cuh"
 #include "router.cuh"
 
 namespace {
@@ -368,6 +369,56 @@ moe_status moe_combine(const void* y_disp, int dtype, const float* topk_w, const
   else
     err = moe::launch_combine((const float*)y_disp, topk_w, slot_to_row, T, k, H, (float*)y, s);
   return cuda_status(err, "moe_combine");
+}
+
+moe_status moe_eplb_plan(const int64_t* load, int E, int R, int slots_per_rank, int32_t* phys_to_logical,
+                         int32_t* replica_offsets, int32_t* replicas) {
+  MOE_REQUIRE(E >= 1 && R >= 1 && slots_per_rank >= 1, "E, R and slots_per_rank must be >= 1");
+  MOE_REQUIRE((long long)R * slots_per_rank <= moe::kEplbMaxSlots, "R * slots_per_rank must be <= 2^20");
+  MOE_REQUIRE(R * slots_per_rank >= E, "R * slots_per_rank must be >= E (every expert needs a slot)");
+  MOE_REQUIRE(load != nullptr && phys_to_logical != nullptr && replica_offsets != nullptr && replicas != nullptr,
+              "moe_eplb_plan: host arrays must not be NULL");
+  for (int e = 0; e < E; ++e)
+    MOE_REQUIRE(load[e] >= 0 && load[e] < moe::kEplbMaxLoad, "loads must be in [0, 2^40)");
+  if (!moe::eplb_plan_host(load, E, R, slots_per_rank, phys_to_logical, replica_offsets, replicas))
+    return fail(MOE_ERR_INVALID_ARG, "moe_eplb_plan: invalid sizes");
+  return MOE_OK;
+}
+
+moe_status moe_eplb_remap(const int32_t* topk_ids, int T, int k, int E, const int32_t* replica_offsets,
+                          const int32_t* replicas, int P, int32_t* phys_ids, void* stream) {
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  MOE_REQUIRE(k >= 1 && k <= 8, "k must be in [1, 8]");
+  MOE_REQUIRE(E >= 1 && P >= E && P <= moe::kEplbMaxSlots, "need 1 <= E <= P <= 2^20");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
+  MOE_REQUIRE_PTR(replica_offsets, 4, "replica_offsets");
+  MOE_REQUIRE_PTR(replicas, 4, "replicas");
+  MOE_REQUIRE_PTR(phys_ids, 4, "phys_ids");
+  return cuda_status(moe::launch_eplb_remap(topk_ids, T, k, E, replica_offsets, replicas, P, phys_ids,
+                                            (cudaStream_t)stream),
+                     "moe_eplb_remap");
+}
+
+moe_status moe_eplb_replicate(const void* w, size_t expert_bytes, int E, const int32_t* phys_to_logical, int P,
+                              void* w_phys, void* stream) {
+  MOE_REQUIRE(E >= 1 && P >= 1, "E and P must be >= 1");
+  MOE_REQUIRE(phys_to_logical != nullptr, "phys_to_logical (host array) must not be NULL");
+  for (int p = 0; p < P; ++p)
+    MOE_REQUIRE(phys_to_logical[p] >= 0 && phys_to_logical[p] < E, "phys_to_logical entries must be in [0, E)");
+  if (expert_bytes == 0) return MOE_OK;
+  MOE_REQUIRE(w != nullptr && w_phys != nullptr, "w and w_phys must not be NULL");
+  const char* src = static_cast<const char*>(w);
+  char* dst = static_cast<char*>(w_phys);
+  MOE_REQUIRE(dst + (size_t)P * expert_bytes <= src || src + (size_t)E * expert_bytes <= dst,
+              "w and w_phys must not overlap");
+  for (int p = 0; p < P; ++p) {
+    cudaError_t err = cudaMemcpyAsync(dst + (size_t)p * expert_bytes, src + (size_t)phys_to_logical[p] * expert_bytes,
+                                      expert_bytes, cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+    if (err != cudaSuccess) return cuda_status(err, "moe_eplb_replicate");
+  }
+  return MOE_OK;
 }
 
 moe_status moe_selftest_wait_timeout(unsigned int limit_us, void* stream) {
