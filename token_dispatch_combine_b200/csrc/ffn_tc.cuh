@@ -273,11 +273,16 @@ struct Params {
 // ---- A-row gather (dispatch fused into the gate/up projection)
 // kGatherThreads extra threads per CTA copy the A tile rows of each k-block
 // from x with 16-byte cp.async: thread t owns 16-byte chunk c = t % 8 of rows
-// t / 8 + 16 j (j < 8) of the 128-row tile, written to its 128-byte
+// t / 8 + (kGatherThreads / 8) j of the 128-row tile, written to its 128-byte
 // swizzled position (chunk c ^ (row % 8)).  Each thread then arrives on the
 // stage's full barrier when its copies land (cp.async.mbarrier.arrive.noinc).
-constexpr int kGatherThreads = 128;
-constexpr int kGatherRowsPerThread = 8;
+#ifndef MOE_TC_GATHER_THREADS
+#define MOE_TC_GATHER_THREADS 128
+#endif
+constexpr int kGatherThreads = MOE_TC_GATHER_THREADS;       // 32, 64 or 128
+constexpr int kGatherRowStep = kGatherThreads / 8;          // rows between a thread's rows
+constexpr int kGatherRowsPerThread = 128 / kGatherRowStep;  // 8 at 128 threads
+static_assert(kGatherThreads == 32 || kGatherThreads == 64 || kGatherThreads == 128, "gather threads");
 
 // Slots (row_to_slot entries) of this thread's rows of the tile [r0, r_end),
 // -1 for rows past r_end.  Loaded one tile ahead, so their latency hides
@@ -287,7 +292,7 @@ __device__ __forceinline__ void gather_load_slots(const Params& p, int r0, int r
   const int rr = gt >> 3;
 #pragma unroll
   for (int j = 0; j < kGatherRowsPerThread; ++j) {
-    const int r = r0 + rr + 16 * j;
+    const int r = r0 + rr + kGatherRowStep * j;
     slot[j] = r < r_end ? __ldg(p.gather_rows + r) : -1;
   }
 }
@@ -301,11 +306,11 @@ __device__ __forceinline__ void gather_load_slots(const Params& p, int r0, int r
 __device__ __forceinline__ int gather_rows_of_thread(const Params& p, const int (&slot)[kGatherRowsPerThread], int gt,
                                                      const char* (&src)[kGatherRowsPerThread],
                                                      uint32_t (&dst_off)[kGatherRowsPerThread]) {
-  const int c = gt & 7, rr = gt >> 3;  // chunk, first row (0..15)
+  const int c = gt & 7, rr = gt >> 3;  // chunk, first row (0 .. kGatherRowStep - 1)
   int n = 0;
 #pragma unroll
   for (int j = 0; j < kGatherRowsPerThread; ++j) {
-    const int row = rr + 16 * j;
+    const int row = rr + kGatherRowStep * j;
     src[j] = nullptr;
     dst_off[j] = (uint32_t)row * 128u + (uint32_t)((c ^ (row & 7)) << 4);
     if (slot[j] != -1) {
