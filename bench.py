@@ -467,7 +467,8 @@ def run_ours(args, wl):
             "remap_us": statistics.median(a.elapsed_time(b) for a, b in ev_r) * 1e3,
             "balanced_step_ms": statistics.median(c.elapsed_time(d) for c, d in ev_s),
             "note": "plan from the warm-up's expert counts; a replica has its expert's weights, so outputs "
-                    "are unchanged; on one GPU the ranks are logical, so the step time shows the remap's cost",
+                    "are unchanged; on one GPU the ranks are logical, so the balanced step shows only costs: "
+                    "the remap and the extra partial GEMM tiles of more (physical) experts",
         }
         del bal
     step_ms, dc_pair_ms, dc_stream_ms, t_disp_rows, t_comb_rows, *stage_max = max_over_ranks(
