@@ -31,6 +31,10 @@ def test_library_exports_every_declared_symbol():
     for name in declared_functions():
         assert hasattr(lib, name), name
     assert set(_native.EXPORTS) <= set(declared_functions())
+    # and the binding configures every declared call (argument and result types)
+    assert set(declared_functions()) <= set(_native.EXPORTS)
+    for name in declared_functions():
+        assert getattr(lib, name).restype is not None, name
 
 
 def test_version_and_status_strings():
