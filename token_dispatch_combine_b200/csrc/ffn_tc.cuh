@@ -57,6 +57,12 @@
 #ifndef MOE_TC_GROUP_M
 #define MOE_TC_GROUP_M 16
 #endif
+//  MOE_TC_EXPERT_GROUPS: raster groups end at expert boundaries (whole experts
+//    until a group holds at least the group size in m-tiles) instead of every
+//    group-size m-tiles, so an expert's m-tiles are never split across groups.
+#ifndef MOE_TC_EXPERT_GROUPS
+#define MOE_TC_EXPERT_GROUPS 1
+#endif
 #ifndef MOE_TC_HINT_A
 #define MOE_TC_HINT_A 0
 #endif
@@ -361,7 +367,7 @@ struct Cfg {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr size_t smem_bytes(int E) {
     return 1024 /* alignment slack */ + (size_t)STAGES * kStageBytes + 256 /* barriers etc */ +
-           sizeof(int32_t) * 2 * ((size_t)E + 1);
+           sizeof(int32_t) * (3 * ((size_t)E + 1) + 1);
   }
   static_assert(MMA_N % 16 == 0 && MMA_N >= 16 && MMA_N <= 256, "UMMA N for M=128");
   static_assert(!GATEUP || BN % 64 == 0, "gate/up halves must be whole 64-column boxes");
@@ -382,6 +388,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int32_t* s_seg = reinterpret_cast<int32_t*>(smem + (size_t)STAGES * C::kStageBytes + 256);  // [E + 1]
   int32_t* s_pre = s_seg + (p.E + 1);                                                         // [E + 1]
+  int32_t* s_grp = s_pre + (p.E + 1);  // [E + 2]: raster group starts (m-tiles), count at [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = (int)lane_id();
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -450,6 +457,24 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
       run += (s_seg[e + 1] - s_seg[e] + BM - 1) / BM;
     }
     if (lane == 31) s_pre[E] = incl;
+    if (MOE_TC_EXPERT_GROUPS) {
+      // raster groups of whole experts: experts in order until a group holds at
+      // least MOE_TC_GROUP_M m-tiles, so that no expert's weights are streamed twice
+      __syncwarp();
+      if (lane == 0) {
+        int ng = 0, start = 0;
+        s_grp[0] = 0;
+        for (int e = 0; e < E; ++e) {
+          const int end = s_pre[e + 1];
+          if (end - start >= MOE_TC_GROUP_M) {
+            s_grp[++ng] = end;
+            start = end;
+          }
+        }
+        if (start < s_pre[E]) s_grp[++ng] = s_pre[E];
+        s_grp[E + 1] = ng;
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -462,7 +487,19 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
   // tile -> (expert, first row, end row, first output column)
   auto tile_coords = [&](int tile, int& e, int& m0, int& mend, int& n0) {
     int mt, nt;
-    if (MOE_TC_GROUP_M > 0) {
+    if (MOE_TC_EXPERT_GROUPS) {
+      // group g: m-tiles [s_grp[g], s_grp[g + 1]), n-tile-major inside
+      int lo = 0, hi = s_grp[p.E + 1] - 1;  // largest g with s_grp[g] * ntn <= tile
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_grp[mid] * p.ntn <= tile) lo = mid;
+        else hi = mid - 1;
+      }
+      const int gm0 = s_grp[lo], gm = s_grp[lo + 1] - gm0;
+      const int r = tile - gm0 * p.ntn;
+      nt = r / gm;
+      mt = gm0 + (r - nt * gm);
+    } else if (MOE_TC_GROUP_M > 0) {
       // groups of MOE_TC_GROUP_M m-tiles; inside a group, n-tile-major
       const int per_group = MOE_TC_GROUP_M * p.ntn;
       const int g = tile / per_group, r = tile - g * per_group;

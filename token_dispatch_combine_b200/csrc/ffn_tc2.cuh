@@ -131,7 +131,7 @@ struct Cfg2 {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;  // per CTA
   static constexpr int STAGES = 6;
   static constexpr size_t smem_bytes(int E) {
-    return 1024 + (size_t)STAGES * kStageBytes + 256 + sizeof(int32_t) * 2 * ((size_t)E + 1);
+    return 1024 + (size_t)STAGES * kStageBytes + 256 + sizeof(int32_t) * (3 * ((size_t)E + 1) + 1);
   }
 };
 
@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int32_t* s_seg = reinterpret_cast<int32_t*>(smem + (size_t)STAGES * C::kStageBytes + 256);
   int32_t* s_pre = s_seg + (p.E + 1);
+  int32_t* s_grp = s_pre + (p.E + 1);  // [E + 2]: raster group starts (m-tiles), count at [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = (int)lane_id();
   const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs), 1: peer
@@ -223,6 +224,24 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
       run += (s_seg[e + 1] - s_seg[e] + BM2 - 1) / BM2;
     }
     if (lane == 31) s_pre[E] = incl;
+    if (MOE_TC_EXPERT_GROUPS) {
+      // raster groups of whole experts: experts in order until a group holds at
+      // least MOE_TC2_GROUP_M m-tiles, so that no expert's weights are streamed twice
+      __syncwarp();
+      if (lane == 0) {
+        int ng = 0, start = 0;
+        s_grp[0] = 0;
+        for (int e = 0; e < E; ++e) {
+          const int end = s_pre[e + 1];
+          if (end - start >= MOE_TC2_GROUP_M) {
+            s_grp[++ng] = end;
+            start = end;
+          }
+        }
+        if (start < s_pre[E]) s_grp[++ng] = s_pre[E];
+        s_grp[E + 1] = ng;
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -235,7 +254,19 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
   auto tile_coords = [&](int tile, int& e, int& m0, int& mend, int& n0) {
     int mt, nt;
     const int total_mtiles = s_pre[p.E];
-    if (MOE_TC2_GROUP_M > 0) {
+    if (MOE_TC_EXPERT_GROUPS) {
+      // group g: m-tiles [s_grp[g], s_grp[g + 1]), n-tile-major inside
+      int lo = 0, hi = s_grp[p.E + 1] - 1;  // largest g with s_grp[g] * ntn <= tile
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_grp[mid] * p.ntn <= tile) lo = mid;
+        else hi = mid - 1;
+      }
+      const int gm0 = s_grp[lo], gm = s_grp[lo + 1] - gm0;
+      const int r = tile - gm0 * p.ntn;
+      nt = r / gm;
+      mt = gm0 + (r - nt * gm);
+    } else if (MOE_TC2_GROUP_M > 0) {
       const int per_group = MOE_TC2_GROUP_M * p.ntn;
       const int g = tile / per_group, r = tile - g * per_group;
       const int gm = min(MOE_TC2_GROUP_M, total_mtiles - g * MOE_TC2_GROUP_M);
