@@ -99,15 +99,16 @@ def test_gather_bad_slot_is_flagged(name, ffn_tiling):
     wl = CASES[name]
     layer = DeviceLayer(wl)
     ref, rt = run_pair(layer)
-    rts = rt.disp.row_to_slot.clone()
-    rts[0] = -5
-    rts[1] = wl.T * wl.k + 3
-    h = torch.zeros_like(rt.h)
-    moe_ffn_gate_up_gather(layer.x_dev, rts, wl.k, layer.w_gate, layer.w_up, rt.disp.expert_offsets, h)
-    st, bits = moe_get_error()
-    assert st == MOE_ERR_DEVICE and bits & ERR_BAD_ROW
     n = int(ref.disp.expert_offsets[-1])
-    assert torch.equal(h[2:n], ref.h[2:n])  # every other row is unaffected
+    for bad in (-5, -1, wl.T * wl.k + 3):  # -1 included: it must not pass for "no row"
+        rts = rt.disp.row_to_slot.clone()
+        rts[0] = bad
+        rts[1] = wl.T * wl.k + 3
+        h = torch.zeros_like(rt.h)
+        moe_ffn_gate_up_gather(layer.x_dev, rts, wl.k, layer.w_gate, layer.w_up, rt.disp.expert_offsets, h)
+        st, bits = moe_get_error()
+        assert st == MOE_ERR_DEVICE and bits & ERR_BAD_ROW, bad
+        assert torch.equal(h[2:n], ref.h[2:n])  # every other row is unaffected
     assert moe_get_error() == (0, 0)  # the word was cleared
 
 

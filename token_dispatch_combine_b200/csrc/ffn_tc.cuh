@@ -47,6 +47,8 @@
 
 #include <cuda.h>
 
+#include <climits>
+
 #include "common.cuh"
 
 // Tuning knobs (compile-time).
@@ -291,15 +293,16 @@ constexpr int kGatherRowsPerThread = 128 / kGatherRowStep;  // 8 at 128 threads
 static_assert(kGatherThreads == 32 || kGatherThreads == 64 || kGatherThreads == 128, "gather threads");
 
 // Slots (row_to_slot entries) of this thread's rows of the tile [r0, r_end),
-// -1 for rows past r_end.  Loaded one tile ahead, so their latency hides
-// behind the previous tile's k-blocks.
+// kNoGatherRow for rows past r_end.  Loaded one tile ahead, so their latency
+// hides behind the previous tile's k-blocks.
+constexpr int kNoGatherRow = INT_MIN;
 __device__ __forceinline__ void gather_load_slots(const Params& p, int r0, int r_end, int gt,
                                                   int (&slot)[kGatherRowsPerThread]) {
   const int rr = gt >> 3;
 #pragma unroll
   for (int j = 0; j < kGatherRowsPerThread; ++j) {
     const int r = r0 + rr + kGatherRowStep * j;
-    slot[j] = r < r_end ? __ldg(p.gather_rows + r) : -1;
+    slot[j] = r < r_end ? __ldg(p.gather_rows + r) : kNoGatherRow;
   }
 }
 
@@ -319,7 +322,7 @@ __device__ __forceinline__ int gather_rows_of_thread(const Params& p, const int 
     const int row = rr + kGatherRowStep * j;
     src[j] = nullptr;
     dst_off[j] = (uint32_t)row * 128u + (uint32_t)((c ^ (row & 7)) << 4);
-    if (slot[j] != -1) {
+    if (slot[j] != kNoGatherRow) {
       int t = slot[j] / p.gather_k;
       if (slot[j] < 0 || t >= p.gather_T) {
         flag_error(kErrBadRow);
