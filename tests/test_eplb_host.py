@@ -87,3 +87,34 @@ def test_remap_and_replicate_reject_on_the_host():
     p2l = np.array([0, 1, 2], np.int32)
     assert lib.moe_eplb_replicate(FAKE, 64, 8, p2l.ctypes.data, 3, FAKE + 64, None) == _native.MOE_ERR_INVALID_ARG
     assert b"overlap" in lib.moe_last_error_message()
+
+
+def test_plan_with_loads_near_the_limit_matches_oracle():
+    """Loads up to 2^40 - 1 with up to thousands of replicas: load * n stays below 2^63 in both
+    implementations and they still agree exactly; 2^40 itself is rejected."""
+    rng = np.random.default_rng(7)
+    E, R, slots = 64, 16, 200  # 3200 slots: experts get up to hundreds of replicas
+    load = rng.integers(0, 1 << 40, E, dtype=np.int64)
+    load[5] = (1 << 40) - 1
+    load[9] = 0
+    got = lib_plan(load, R, slots)
+    ref = oracle.eplb_plan(load, R, slots)
+    assert got.replicas.tolist() == ref["replicas"].tolist()
+    assert got.phys_to_logical.tolist() == ref["phys_to_logical"].tolist()
+    load[3] = 1 << 40
+    with pytest.raises(Exception):
+        lib_plan(load, R, slots)
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_plan_random_sizes_match_oracle(seed):
+    rng = np.random.default_rng(1000 + seed)
+    R = int(rng.integers(1, 9))
+    E = int(rng.integers(1, 65))
+    slots = int(rng.integers(-(-E // R), -(-E // R) + 4))  # ceil(E / R) .. + 3 spare slots per rank
+    load = rng.integers(0, 10 ** int(rng.integers(1, 7)), E).astype(np.int64)
+    got = lib_plan(load, R, slots)
+    ref = oracle.eplb_plan(load, R, slots)
+    assert got.phys_to_logical.tolist() == ref["phys_to_logical"].tolist()
+    assert got.replica_offsets.tolist() == ref["replica_offsets"].tolist()
+    assert got.replicas.tolist() == ref["replicas"].tolist()
