@@ -430,6 +430,29 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         router_ms = sum(a.elapsed_time(b) for a, b in rev) / args.steps
         del w_router, r_ids, r_w
+    # The whole step replayed from a CUDA graph (one launch from the host per step), L2 flushed
+    # before each replay outside the graph.
+    graph_ms, graph_err = None, None
+    try:
+        g = rt.capture(x, logits, wg, wu, wd)
+        g.replay()
+        torch.cuda.synchronize()
+        ev_g = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        for a, b in ev_g:
+            flush_and_hold()
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = statistics.median(a.elapsed_time(b) for a, b in ev_g)
+        del g
+    except Exception as exc:  # reported in the line; the eager numbers stand on their own
+        graph_err = f"{type(exc).__name__}: {exc}"[:200]
+    st, bits = moe_get_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {bits} in the graph replay")
+
     # Expert placement with replicas (one spare physical slot per logical rank), planned on the
     # warm-up's expert counts: the busiest rank's rows before and after, the remap kernel's time,
     # and the whole balanced step (route, remap, dispatch, FFN, combine over the replicas).
@@ -572,6 +595,8 @@ def run_ours(args, wl):
                 "router_topk_timing": "moe_router_topk (logits = x W_r^T + bias, then top-k), L2 flushed, "
                                       "events per call; bytes T*H*2 + E*H*2 + T*k*8"}),
             **({} if eplb is None else {"eplb": eplb}),
+            "graph_replay_ms": graph_ms,
+            **({} if graph_err is None else {"graph_replay_error": graph_err}),
             "ffn_tiling": {"gate_up": "pair" if tiling == FFN_TILING_PAIR else "single",
                            "down": "pair" if tiling_down == FFN_TILING_PAIR else "single"},
         },
