@@ -202,3 +202,18 @@ def test_router_topk_rejects(kw, needle):
 def test_router_topk_zero_tokens_is_a_host_no_op():
     # T = 0 returns before any pointer is read or any launch
     assert _native.lib().moe_router_topk(None, None, None, 0, 64, 32, 4, None, None, None, None) == 0
+
+
+def test_round_trip_gathers_where_the_ffn_streams_weights():
+    """MoERoundTrip(gather="auto") fuses the row scatter into the gate/up projection only for bf16
+    layers with fewer than 384 rows per expert (host rule, no device needed)."""
+    import torch
+    from token_dispatch_combine_b200 import MoERoundTrip
+    rule = MoERoundTrip.gathers_by_default
+    bf16, f32 = torch.bfloat16, torch.float32
+    assert not rule(4096, 4, 32, bf16)        # GPT-OSS layer, 512 rows per expert: tensor-bound
+    assert rule(8192, 8, 256, bf16)           # DeepSeek-R1 prefill, 256 rows per expert
+    assert rule(128, 8, 256, bf16)            # decode
+    assert rule(383 * 32 // 4, 4, 32, bf16)   # just under 384 rows per expert
+    assert not rule(384 * 32 // 4, 4, 32, bf16)
+    assert not rule(128, 8, 256, f32)         # float32 layers keep the row-moving dispatch

@@ -245,12 +245,17 @@ class MoERoundTrip:
 
     GATHER_MAX_ROWS_PER_EXPERT = 384
 
+    @classmethod
+    def gathers_by_default(cls, T, k, E, dtype) -> bool:
+        """gather="auto": bf16 layers with fewer than GATHER_MAX_ROWS_PER_EXPERT rows per expert."""
+        return dtype == torch.bfloat16 and T * k < cls.GATHER_MAX_ROWS_PER_EXPERT * E
+
     def __init__(self, T, H, I, E, k, R, dtype, device="cuda", src_counts=True, gather="auto"):
         self.T, self.H, self.I, self.E, self.k, self.R = T, H, I, E, k, R
         self.dtype = dtype
         self.device = torch.device(device)
         if gather == "auto":
-            gather = dtype == torch.bfloat16 and T * k < self.GATHER_MAX_ROWS_PER_EXPERT * E
+            gather = self.gathers_by_default(T, k, E, dtype)
         self.gather = bool(gather)
         self._x = None
         S = T * k
