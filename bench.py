@@ -627,7 +627,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="gptoss_uniform", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--config", default="gptoss_uniform", choices=sorted(synth.WORKLOADS) + sorted(synth.PROFILE_WORKLOADS),
+                    help="benchmark layer (or a profiling case: a small layer of the same shapes)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ffn-tiling", default="auto", choices=["auto", "single", "pair"],
                     help="tile shape of the bf16 expert FFN (moe_set_ffn_tiling); auto picks by rows per expert")
@@ -639,7 +640,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    wl = synth.WORKLOADS[args.config]
+    wl = synth.WORKLOADS.get(args.config) or synth.PROFILE_WORKLOADS[args.config]
     if args.impl == "reference":
         return run_reference(args, wl)
     rc = run_ours(args, wl)

@@ -177,3 +177,11 @@ WORKLOADS = {
                              bias="normal0.5"),
     "dsr1_decode": Workload("dsr1_decode", T=128, H=7168, I=2048, E=256, k=8, R=32, dtype="bf16", seed=4),
 }
+
+# Profiling cases (not benchmark layers): the DeepSeek-R1 prefill layer's shapes with 32 experts,
+# so that a multi-pass profiler capture holds a few GB (256 rows per expert on average, the same
+# routing bias and seed).
+PROFILE_WORKLOADS = {
+    "dsr1_prefill_slice": Workload("dsr1_prefill_slice", T=1024, H=7168, I=2048, E=32, k=8, R=8, dtype="bf16",
+                                   seed=3, bias="normal0.5"),
+}
