@@ -14,6 +14,12 @@
  *   moe_combine    gather each token's k expert outputs, weight them by the
  *                  router weights, sum, and write them in original token order
  *
+ * and, beside them: moe_router_topk (router affinities on tensor cores fused
+ * with the top-k), an index-only moe_dispatch with moe_ffn_gate_up_gather /
+ * moe_expert_ffn_gather (the row scatter fused into the gate/up projection),
+ * and moe_eplb_plan / moe_eplb_remap / moe_eplb_replicate (replicas of hot
+ * experts placed over the logical ranks).
+ *
  * Sources (page title, section):
  *  [EPRT]   "EP: Partition Experts and Route Tokens": "Send tokens to experts
  *           and return their results" (route, dispatch, per-expert batched
@@ -32,10 +38,12 @@
  *  - T tokens, H hidden, I intermediate, E experts, k experts per token
  *    (1 <= k <= min(E, 8)), R logical EP ranks (E % R == 0), S = T*k slots.
  *    Slot s = t*k + j is token t's j-th choice.
- *  - All array arguments are DEVICE pointers owned by the caller, row-major;
- *    activation and weight buffers (and the workspace) 16-byte aligned,
- *    int32/float32 index and weight arrays 4-byte aligned.  The library never allocates, frees or copies to the
- *    host, and never synchronises, except moe_get_error.
+ *  - All array arguments are DEVICE pointers owned by the caller, row-major,
+ *    except where a call says HOST (moe_eplb_plan's arrays, the
+ *    phys_to_logical table of moe_eplb_replicate); activation and weight
+ *    buffers (and the workspace) 16-byte aligned, int32/float32 index and
+ *    weight arrays 4-byte aligned.  The library never allocates, frees or
+ *    copies to the host, and never synchronises, except moe_get_error.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
  *    enqueued asynchronously on it.
  *  - Invalid arguments are rejected on the host before anything is enqueued
