@@ -53,6 +53,9 @@ def _configure(lib):
     lib.oracle_eplb_plan.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     lib.oracle_eplb_plan.restype = i32
     lib.oracle_eplb_remap.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    lib.oracle_rank_partials.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
+    lib.oracle_rank_partials.restype = i32
+    lib.oracle_reduce_ranks.argtypes = [vp, i32, i32, i32, vp]
     return lib
 
 
@@ -208,6 +211,32 @@ def combine(y_disp: np.ndarray, topk_w: np.ndarray, slot_to_row: np.ndarray) -> 
     H = y_disp.shape[1]
     y = np.empty((T, H), np.float64)
     _get().oracle_combine(y_disp.ctypes.data, topk_w.ctypes.data, s2r.ctypes.data, T, k, H, y.ctypes.data)
+    return y
+
+
+def rank_partials(y_disp: np.ndarray, topk_w: np.ndarray, topk_ids: np.ndarray, slot_to_row: np.ndarray, E: int,
+                  R: int) -> np.ndarray:
+    """Masking form: part[r][t] = sum of w[t,j] * y_disp[slot_to_row[t*k+j]] over the choices j of
+    token t whose expert sits on rank r (experts [r*E/R, (r+1)*E/R)); [R, T, H] float64."""
+    y_disp = _c(y_disp, np.float64)
+    topk_w = _c(topk_w, np.float32)
+    ids = _c(topk_ids, np.int32)
+    s2r = _c(slot_to_row, np.int32)
+    T, k = topk_w.shape
+    H = y_disp.shape[1]
+    part = np.empty((R, T, H), np.float64)
+    if _get().oracle_rank_partials(y_disp.ctypes.data, topk_w.ctypes.data, ids.ctypes.data, s2r.ctypes.data, T, k,
+                                   H, E, R, part.ctypes.data) != 0:
+        raise ValueError("oracle_rank_partials: bad sizes")
+    return part
+
+
+def reduce_ranks(part: np.ndarray) -> np.ndarray:
+    """y[t] = sum over ranks r (ascending) of part[r][t], float64."""
+    part = _c(part, np.float64)
+    R, T, H = part.shape
+    y = np.empty((T, H), np.float64)
+    _get().oracle_reduce_ranks(part.ctypes.data, T, H, R, y.ctypes.data)
     return y
 
 

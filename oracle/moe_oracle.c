@@ -261,6 +261,49 @@ void oracle_combine(const double* y_disp, const float* topk_w, const int32_t* sl
   }
 }
 
+/* ------------------------------------------------ masking: rank partials
+ * [NEURON] "Collective Patterns / Prefill (CTE kernel)", steps 5-6, and "Why
+ * a Single All-Reduce/Reduce-Scatter Works": in the masking form every rank
+ * runs all T tokens against its own experts only, and a token none of whose
+ * chosen experts sit on rank r gets zeros from r ("Tokens not routed to a
+ * rank's experts produce zero output").  With rank r owning experts
+ * [r*E/R, (r+1)*E/R) ("Limitations" 3-4), rank r's partial output is
+ *   part[r][t] = sum over j (ascending) with ids[t*k+j] / (E/R) == r of
+ *                w[t*k+j] * y_disp[slot_to_row[t*k+j]],
+ * the expert output of each slot weighted by its affinity.  Slots with
+ * slot_to_row < 0 (dropped) contribute nothing.  part is [R][T][H], float64.
+ * Returns 0, or -1 for bad sizes. */
+int oracle_rank_partials(const double* y_disp, const float* topk_w, const int32_t* ids,
+                         const int32_t* slot_to_row, int T, int k, int H, int E, int R, double* part) {
+  if (T < 0 || k < 1 || H < 1 || E < 1 || R < 1 || E % R != 0) return -1;
+  const int EL = E / R;
+  for (int r = 0; r < R; ++r) {
+    for (int t = 0; t < T; ++t) {
+      double* out = part + ((size_t)r * T + t) * H;
+      for (int h = 0; h < H; ++h) out[h] = 0.0;
+      for (int j = 0; j < k; ++j) {
+        const int s = t * k + j, e = ids[s], row = slot_to_row[s];
+        if (row < 0 || e < 0 || e >= E || e / EL != r) continue;
+        const double affinity = (double)topk_w[s];
+        for (int h = 0; h < H; ++h) out[h] += affinity * y_disp[(size_t)row * H + h];
+      }
+    }
+  }
+  return 0;
+}
+
+/* The reduction of the masking form (the reduce-scatter of "Collective
+ * Patterns / Prefill", all-reduce in decode): y[t] = sum over r ascending of
+ * part[r][t].  float64. */
+void oracle_reduce_ranks(const double* part, int T, int H, int R, double* y) {
+  for (int t = 0; t < T; ++t)
+    for (int h = 0; h < H; ++h) {
+      double acc = 0.0;
+      for (int r = 0; r < R; ++r) acc += part[((size_t)r * T + t) * H + h];
+      y[(size_t)t * H + h] = acc;
+    }
+}
+
 /* ----------------------------------------------------------------- EPLB
  * [WIKI] "工作机制" / "边界与常见误解" (third point): routing is dynamic, so
  * the per-expert token counts drift and a balancer redistributes hot and

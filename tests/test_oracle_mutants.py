@@ -36,6 +36,9 @@ MUTANTS = {
     "eplb_places_on_heaviest_rank": ("(r_best < 0 || rank_load[r] < rank_load[r_best])",
                                      "(r_best < 0 || rank_load[r] > rank_load[r_best])"),
     "eplb_remap_first_replica_only": ("out = replicas[replica_offsets[e] + t % n];", "out = replicas[replica_offsets[e]];"),
+    "partials_round_robin_owner": ("e / EL != r) continue;", "e % R != r) continue;"),
+    "partials_drop_weight": ("out[h] += affinity * y_disp", "out[h] += y_disp"),
+    "reduce_skips_last_rank": ("for (int r = 0; r < R; ++r) acc += part", "for (int r = 0; r < R - 1; ++r) acc += part"),
     "combine_drops_last_choice": ("for (int j = 0; j < k; ++j) {\n      int row = slot_to_row", "for (int j = 0; j < k - 1; ++j) {\n      int row = slot_to_row"),
 }
 
@@ -59,6 +62,7 @@ PINS = [
     pins.test_eplb_equal_loads_without_extra_slots_alternate_ranks,
     pins.test_eplb_remainders_go_to_the_first_replicas,
     lambda: pins.test_eplb_plan_invariants(20, 4, 6, 3),
+    lambda: pins.test_rank_partials_equal_dense_masked_moe_per_rank(9, 16, 24, 8, 3, 4),
 ]
 
 

@@ -104,6 +104,17 @@ def test_masked_sum_ep8():
         if r not in g["expected"]["contributing_ranks"]:
             assert not parts[-1].any()
     np.testing.assert_allclose(sum(parts), full, rtol=0, atol=1e-12)
+    # The masking form's own functions: a contributing rank holds exactly its expert's output
+    # times its affinity, every other rank exactly zero, and the reduction gives the output.
+    part = oracle.rank_partials(y_disp, w, ids, idx["slot_to_row"], E, R)
+    rows = idx["slot_to_row"]
+    for j, e in enumerate(ids[0]):
+        r = int(e) // EL
+        np.testing.assert_array_equal(part[r, 0], float(w[0, j]) * y_disp[rows[j]])
+    for r in range(R):
+        if r not in g["expected"]["contributing_ranks"]:
+            assert not part[r].any()
+    np.testing.assert_allclose(oracle.reduce_ranks(part), full, rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------------------
@@ -259,6 +270,45 @@ def test_round_trip_equals_dense_masked_moe(T, H, I, E, k, R):
     parts = sum(oracle.combine(out["y_disp"], np.where(out["ids"] // EL == r, out["w"], 0).astype(np.float32),
                                out["slot_to_row"]) for r in range(R))
     np.testing.assert_allclose(parts, out["y"], rtol=0, atol=1e-12)
+
+
+def _dense_moe_rank(x, logits, k, wg, wu, wd, r, EL):
+    """Rank r's output in the masking form, by brute force: every token through every expert
+    of rank r, each masked by the token's top-k softmax weight for that expert (float64)."""
+    T, E = logits.shape
+    y = np.zeros((T, x.shape[1]))
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -logits[t].astype(np.float64)))[:k]
+        sel = logits[t, order].astype(np.float64)
+        p = np.exp(sel - sel.max())
+        p /= p.sum()
+        mask_w = np.zeros(E)
+        mask_w[order] = p
+        for e in range(r * EL, (r + 1) * EL):
+            g = x[t] @ wg[e]
+            u = x[t] @ wu[e]
+            y[t] += mask_w[e] * ((g / (1.0 + np.exp(-g)) * u) @ wd[e])
+    return y
+
+
+@pytest.mark.parametrize("T,H,I,E,k,R", [(12, 8, 12, 4, 2, 2), (9, 16, 24, 8, 3, 4), (7, 8, 16, 6, 6, 3)])
+def test_rank_partials_equal_dense_masked_moe_per_rank(T, H, I, E, k, R):
+    """Each rank's partial output of the masking form equals that rank's experts run densely
+    over all tokens with the top-k mask, and the rank-ordered reduction equals the round trip."""
+    rng = np.random.default_rng(T * 7 + H + E)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    wg = (rng.standard_normal((E, H, I)) / math.sqrt(H)).astype(np.float32)
+    wu = (rng.standard_normal((E, H, I)) / math.sqrt(H)).astype(np.float32)
+    wd = (rng.standard_normal((E, I, H)) / math.sqrt(I)).astype(np.float32)
+    out = oracle.round_trip(x, logits, k, E, R, wg, wu, wd)
+    part = oracle.rank_partials(out["y_disp"], out["w"], out["ids"], out["slot_to_row"], E, R)
+    assert part.shape == (R, T, H)
+    for r in range(R):
+        ref = _dense_moe_rank(x.astype(np.float64), logits, k, wg.astype(np.float64), wu.astype(np.float64),
+                              wd.astype(np.float64), r, E // R)
+        np.testing.assert_allclose(part[r], ref, rtol=1e-5, atol=1e-6)  # weights are float32-rounded
+    np.testing.assert_allclose(oracle.reduce_ranks(part), out["y"], rtol=0, atol=1e-12)
 
 
 def test_ffn_bf16_weights_widen_exactly():
