@@ -56,6 +56,8 @@ def _configure(lib):
     lib.oracle_rank_partials.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     lib.oracle_rank_partials.restype = i32
     lib.oracle_reduce_ranks.argtypes = [vp, i32, i32, i32, vp]
+    lib.oracle_ep_plan.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.oracle_ep_plan.restype = i32
     return lib
 
 
@@ -238,6 +240,87 @@ def reduce_ranks(part: np.ndarray) -> np.ndarray:
     y = np.empty((T, H), np.float64)
     _get().oracle_reduce_ranks(part.ctypes.data, T, H, R, y.ctypes.data)
     return y
+
+
+def ep_plan(topk_ids: np.ndarray, topk_w: np.ndarray, E: int, R: int) -> dict:
+    """Send plan of one source rank in the expert-parallel exchange (oracle_ep_plan): one row per
+    (token, destination rank) holding any of its experts, ordered by destination then token, with
+    the token's local expert ids and weights on that rank.  Keys: send_counts [R], send_offsets
+    [R+1], slot_send_row [T*k], row_token [n], row_ids [n, k], row_w [n, k] (n = send rows)."""
+    ids = _c(topk_ids, np.int32)
+    w = _c(topk_w, np.float32)
+    T, k = ids.shape
+    cnt = np.empty(R, np.int32)
+    off = np.empty(R + 1, np.int32)
+    ssr = np.empty(T * k, np.int32)
+    cap = max(1, T * k)
+    tok = np.empty(cap, np.int32)
+    rid = np.empty((cap, k), np.int32)
+    rw = np.empty((cap, k), np.float32)
+    n = _get().oracle_ep_plan(ids.ctypes.data, w.ctypes.data, T, k, E, R, cnt.ctypes.data, off.ctypes.data,
+                              ssr.ctypes.data, tok.ctypes.data, rid.ctypes.data, rw.ctypes.data)
+    if n < 0:
+        raise ValueError("oracle_ep_plan: bad sizes")
+    return dict(send_counts=cnt, send_offsets=off, slot_send_row=ssr, row_token=tok[:n].copy(),
+                row_ids=rid[:n].copy(), row_w=rw[:n].copy())
+
+
+def ep_round_trip(xs, logits_list, k: int, E: int, R: int, w_gate, w_up, w_down) -> dict:
+    """The expert-parallel round trip over R source ranks on the CPU: each rank routes its own
+    tokens and plans its sends (ep_plan); destination d receives the rows of sources 0..R-1 in
+    turn (each source's rows for d in its send order), runs each row through its local experts
+    and sums their weighted outputs (one partial per received row); the partials return to
+    their source rows, and each token's output is the sum of its partials over destinations
+    in ascending order.  Returns per-rank lists: plans, received rows / ids / weights / source,
+    partials and outputs y (float64)."""
+    EL = E // R
+    H = xs[0].shape[1]
+    I = w_gate.shape[-1] if isinstance(w_gate, np.ndarray) else next(iter(w_gate.values())).shape[-1]
+    routes = [route(lg, k) for lg in logits_list]
+    plans = [ep_plan(ids, w, E, R) for ids, w in routes]
+    recv_x, recv_ids, recv_w, recv_src, partial = [], [], [], [], []
+    for d in range(R):
+        xr, ir, wr, sr = [], [], [], []
+        for s in range(R):
+            p = plans[s]
+            lo, hi = p["send_offsets"][d], p["send_offsets"][d + 1]
+            xr.append(xs[s][p["row_token"][lo:hi]])
+            ir.append(p["row_ids"][lo:hi])
+            wr.append(p["row_w"][lo:hi])
+            sr.append(np.full(hi - lo, s, np.int32))
+        xr = np.concatenate(xr) if xr else np.zeros((0, H), xs[0].dtype)
+        ir, wr, sr = np.concatenate(ir), np.concatenate(wr), np.concatenate(sr)
+        part = np.zeros((len(xr), H))
+        for i in range(ir.shape[1]):  # choice i of every received row that has one
+            sel = np.nonzero(ir[:, i] >= 0)[0]
+            if len(sel):
+                u = ffn_rows(xr[sel], ir[sel, i] + d * EL, w_gate, w_up, w_down, H, I)
+                part[sel] += wr[sel, i].astype(np.float64)[:, None] * u
+        recv_x.append(xr)
+        recv_ids.append(ir)
+        recv_w.append(wr)
+        recv_src.append(sr)
+        partial.append(part)
+    ys = []
+    for s in range(R):
+        p = plans[s]
+        T = xs[s].shape[0]
+        ret = np.zeros((p["send_offsets"][R], H))
+        for d in range(R):  # rows of source s at destination d come back in send order
+            at = sum(plans[q]["send_counts"][d] for q in range(s))
+            n = p["send_counts"][d]
+            ret[p["send_offsets"][d]:p["send_offsets"][d] + n] = partial[d][at:at + n]
+        y = np.zeros((T, H))
+        ids = routes[s][0]
+        for t in range(T):
+            for d in range(R):
+                rows = [p["slot_send_row"][t * k + j] for j in range(k)
+                        if 0 <= ids[t, j] < E and ids[t, j] // EL == d]
+                if rows:
+                    y[t] += ret[rows[0]]
+        ys.append(y)
+    return dict(routes=routes, plans=plans, recv_x=recv_x, recv_ids=recv_ids, recv_w=recv_w, recv_src=recv_src,
+                partial=partial, y=ys)
 
 
 def round_trip(x: np.ndarray, logits: np.ndarray, k: int, E: int, R: int, w_gate, w_up, w_down):

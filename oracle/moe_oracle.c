@@ -304,6 +304,74 @@ void oracle_reduce_ranks(const double* part, int T, int H, int R, double* y) {
     }
 }
 
+/* ------------------------------------------ expert-parallel exchange plan
+ * [EPRT] "Send tokens to experts and return their results": each GPU routes
+ * its own tokens and sends each token vector to the GPU that holds its
+ * selected expert; destinations receive different counts (an exchange by
+ * destination); results return to their source GPU and original token.
+ * "Return multiple expert results to the same token": input delivery is
+ * shared when two selected experts reside on the same GPU, and the source
+ * forms the weighted sum of the token's results.  [NEURON] "Limitations"
+ * 3-4: rank d holds experts [d*E/R, (d+1)*E/R).
+ *
+ * Plan of one source rank with T tokens (ids [T][k] global expert ids,
+ * w [T][k] weights):
+ *   J(t, d)        = the choices j (ascending) of token t with ids[t][j] on d;
+ *   send_counts[d] = #{t : J(t, d) non-empty}: token t's row goes to d once;
+ *   send rows are ordered by destination, then by token: send_offsets is the
+ *   exclusive prefix sum of send_counts, and the row of (t, d) is
+ *   send_offsets[d] + #{t' < t : J(t', d) non-empty};
+ *   slot_send_row[t*k + j] = that row for d = ids[t][j] / (E/R) (-1 for an
+ *   id outside [0, E));
+ *   row_token[row]          = t;
+ *   row_ids[row][i], row_w[row][i] (i < k): for the i-th choice j of J(t, d),
+ *   the expert's local id ids[t][j] - d*E/R and the weight w[t][j]; -1 and 0
+ *   past |J(t, d)|.
+ * Arrays sized for T*k rows (the most there can be).  Returns the number of
+ * send rows, or -1 for bad sizes. */
+int oracle_ep_plan(const int32_t* ids, const float* w, int T, int k, int E, int R, int32_t* send_counts,
+                   int32_t* send_offsets, int32_t* slot_send_row, int32_t* row_token, int32_t* row_ids,
+                   float* row_w) {
+  if (T < 0 || k < 1 || E < 1 || R < 1 || E % R != 0) return -1;
+  const int EL = E / R;
+  for (int d = 0; d < R; ++d) {
+    send_counts[d] = 0;
+    for (int t = 0; t < T; ++t)
+      for (int j = 0; j < k; ++j) {
+        const int e = ids[(size_t)t * k + j];
+        if (e >= 0 && e < E && e / EL == d) {
+          send_counts[d] += 1;
+          break;
+        }
+      }
+  }
+  send_offsets[0] = 0;
+  for (int d = 0; d < R; ++d) send_offsets[d + 1] = send_offsets[d] + send_counts[d];
+  for (int s = 0; s < T * k; ++s) slot_send_row[s] = -1;
+  for (int d = 0; d < R; ++d) {
+    int row = send_offsets[d];
+    for (int t = 0; t < T; ++t) {
+      int n = 0;
+      for (int j = 0; j < k; ++j) {
+        const int e = ids[(size_t)t * k + j];
+        if (e < 0 || e >= E || e / EL != d) continue;
+        row_ids[(size_t)row * k + n] = e - d * EL;
+        row_w[(size_t)row * k + n] = w[(size_t)t * k + j];
+        slot_send_row[(size_t)t * k + j] = row;
+        n += 1;
+      }
+      if (n == 0) continue;
+      for (int i = n; i < k; ++i) {
+        row_ids[(size_t)row * k + i] = -1;
+        row_w[(size_t)row * k + i] = 0.0f;
+      }
+      row_token[row] = t;
+      row += 1;
+    }
+  }
+  return send_offsets[R];
+}
+
 /* ----------------------------------------------------------------- EPLB
  * [WIKI] "工作机制" / "边界与常见误解" (third point): routing is dynamic, so
  * the per-expert token counts drift and a balancer redistributes hot and

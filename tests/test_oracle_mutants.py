@@ -39,6 +39,10 @@ MUTANTS = {
     "partials_round_robin_owner": ("e / EL != r) continue;", "e % R != r) continue;"),
     "partials_drop_weight": ("out[h] += affinity * y_disp", "out[h] += y_disp"),
     "reduce_skips_last_rank": ("for (int r = 0; r < R; ++r) acc += part", "for (int r = 0; r < R - 1; ++r) acc += part"),
+    "ep_no_shared_delivery": ("          send_counts[d] += 1;\n          break;", "          send_counts[d] += 1;"),
+    "ep_rows_in_reverse_token_order": ("    for (int t = 0; t < T; ++t) {\n      int n = 0;",
+                                       "    for (int t = T - 1; t >= 0; --t) {\n      int n = 0;"),
+    "ep_local_id_not_offset": ("row_ids[(size_t)row * k + n] = e - d * EL;", "row_ids[(size_t)row * k + n] = e;"),
     "combine_drops_last_choice": ("for (int j = 0; j < k; ++j) {\n      int row = slot_to_row", "for (int j = 0; j < k - 1; ++j) {\n      int row = slot_to_row"),
 }
 
@@ -63,6 +67,9 @@ PINS = [
     pins.test_eplb_remainders_go_to_the_first_replicas,
     lambda: pins.test_eplb_plan_invariants(20, 4, 6, 3),
     lambda: pins.test_rank_partials_equal_dense_masked_moe_per_rank(9, 16, 24, 8, 3, 4),
+    pins.test_ep_plan_worked_example_top1,
+    pins.test_ep_plan_top2_shares_input_delivery,
+    lambda: pins.test_ep_round_trip_equals_single_gpu_round_trip((9, 3, 6), 16, 8, 6, 3, 3, 1.5),
 ]
 
 

@@ -311,6 +311,81 @@ def test_rank_partials_equal_dense_masked_moe_per_rank(T, H, I, E, k, R):
     np.testing.assert_allclose(oracle.reduce_ranks(part), out["y"], rtol=0, atol=1e-12)
 
 
+def test_ep_plan_worked_example_top1():
+    """The pages' Top-1 round trip as two source ranks: who sends what where, and what each
+    destination receives (A2 goes to GPU 1, B1 to GPU 0, E2 receives A2 and B2)."""
+    g = _load("ep_exchange.json")
+    E, R, c = g["E"], g["R"], g["top1"]
+    ex = c["expected"]
+    plans = []
+    for s in range(R):
+        ids = np.array(c["ids"][s], np.int32)
+        p = oracle.ep_plan(ids, np.ones_like(ids, np.float32), E, R)
+        for key in ("send_counts", "send_offsets", "slot_send_row", "row_token", "row_ids"):
+            assert p[key].tolist() == ex[key][s], (s, key)
+        plans.append(p)
+    # destination d receives sources 0..R-1 in turn: rank 0 gets A1, B1; rank 1 gets A2, B2
+    names = "AB"
+    for d in range(R):
+        got = []
+        for s in range(R):
+            lo, hi = plans[s]["send_offsets"][d], plans[s]["send_offsets"][d + 1]
+            got += [[names[s], int(t)] for t in plans[s]["row_token"][lo:hi]]
+        assert got == ex["received_tokens"][d]
+
+
+def test_ep_plan_top2_shares_input_delivery():
+    """A2's two results come from two GPUs (one row to each); A3's two experts share GPU 1,
+    so its row goes there once and carries both local experts: 3 rows for 4 choices."""
+    g = _load("ep_exchange.json")
+    c = g["top2_shared"]
+    ex = c["expected"]
+    E, R = g["E"], g["R"]
+    logits = np.full((2, E), -30.0, np.float32)
+    logits[0, 0], logits[0, 2] = math.log(7 / 3), 0.0
+    logits[1, 2], logits[1, 3] = math.log(3 / 2), 0.0
+    ids, w = oracle.route(logits, c["k"])
+    assert ids.tolist() == c["ids"]
+    np.testing.assert_allclose(w, c["w"], atol=1e-6, rtol=0)
+    p = oracle.ep_plan(ids, w, E, R)
+    for key in ("send_counts", "send_offsets", "slot_send_row", "row_token", "row_ids"):
+        assert p[key].tolist() == ex[key], key
+    np.testing.assert_allclose(p["row_w"], ex["row_w"], atol=1e-6, rtol=0)
+    assert len(p["row_token"]) == ex["rows_sent_for_four_choices"]
+
+
+def _ep_case(sizes, H, I, E, k, R, seed, bias=0.0):
+    rng = np.random.default_rng(seed)
+    xs = [rng.standard_normal((T, H)).astype(np.float32) for T in sizes]
+    lg = [rng.standard_normal((T, E)).astype(np.float32) for T in sizes]
+    for a in lg:
+        a[:, :E // R] += bias  # experts of rank 0 hot: many tokens share delivery there
+    wg = (rng.standard_normal((E, H, I)) / math.sqrt(H)).astype(np.float32)
+    wu = (rng.standard_normal((E, H, I)) / math.sqrt(H)).astype(np.float32)
+    wd = (rng.standard_normal((E, I, H)) / math.sqrt(I)).astype(np.float32)
+    return xs, lg, wg, wu, wd
+
+
+@pytest.mark.parametrize("sizes,H,I,E,k,R,bias", [((5, 7), 8, 12, 4, 2, 2, 0.0), ((9, 3, 6), 16, 8, 6, 3, 3, 1.5),
+                                                  ((4, 4, 4, 4), 8, 8, 8, 4, 4, 2.0), ((6, 0), 8, 8, 4, 1, 2, 0.0)])
+def test_ep_round_trip_equals_single_gpu_round_trip(sizes, H, I, E, k, R, bias):
+    """The exchange over R source ranks gives each token the output the one-GPU round trip gives
+    it (tokens of all ranks concatenated in rank order), and the plan's invariants hold: one row
+    per (token, destination holding any of its experts), every choice carried exactly once."""
+    xs, lg, wg, wu, wd = _ep_case(sizes, H, I, E, k, R, seed=sum(sizes) + E, bias=bias)
+    ep = oracle.ep_round_trip(xs, lg, k, E, R, wg, wu, wd)
+    ref = oracle.round_trip(np.concatenate(xs), np.concatenate(lg), k, E, R, wg, wu, wd)
+    np.testing.assert_allclose(np.concatenate(ep["y"]), ref["y"], rtol=0, atol=1e-12 * max(1.0, np.abs(ref["y"]).max()))
+    EL = E // R
+    for s, (p, (ids, w)) in enumerate(zip(ep["plans"], ep["routes"])):
+        pairs = {(t, int(e) // EL) for t in range(ids.shape[0]) for e in ids[t]}
+        assert int(p["send_offsets"][-1]) == len(pairs)
+        carried = sorted((int(p["row_token"][r]), int(p["row_ids"][r, i]) + EL * d)
+                         for d in range(R) for r in range(p["send_offsets"][d], p["send_offsets"][d + 1])
+                         for i in range(k) if p["row_ids"][r, i] >= 0)
+        assert carried == sorted((t, int(e)) for t in range(ids.shape[0]) for e in ids[t])
+
+
 def test_ffn_bf16_weights_widen_exactly():
     rng = np.random.default_rng(5)
     H, I, E = 16, 24, 2
