@@ -17,8 +17,10 @@
  * and, beside them: moe_router_topk (router affinities on tensor cores fused
  * with the top-k), an index-only moe_dispatch with moe_ffn_gate_up_gather /
  * moe_expert_ffn_gather (the row scatter fused into the gate/up projection),
- * and moe_eplb_plan / moe_eplb_remap / moe_eplb_replicate (replicas of hot
- * experts placed over the logical ranks).
+ * moe_eplb_plan / moe_eplb_remap / moe_eplb_replicate (replicas of hot
+ * experts placed over the logical ranks), and moe_combine_rank_partials /
+ * moe_reduce_rank_partials (the masking form: per-rank partial outputs and
+ * their rank-ordered sum).
  *
  * Sources (page title, section):
  *  [EPRT]   "EP: Partition Experts and Route Tokens": "Send tokens to experts
@@ -120,8 +122,10 @@ moe_status moe_router_topk(const void* x, const void* w_router, const float* bia
 
 /*
  * Bytes of device workspace moe_dispatch needs for these sizes.  The
- * workspace must be zero-filled once before its first use; each call leaves
- * it ready for the next.  Calls sharing a workspace must not overlap.
+ * workspace must be zero-filled once before its first use; every call leaves
+ * it ready for the next, a call whose grid barrier timed out included (the
+ * last of its CTAs to finish zeroes the barrier's counters).  Calls sharing a
+ * workspace must not overlap.
  */
 size_t moe_dispatch_workspace_bytes(int T, int k, int E, int R);
 
@@ -174,8 +178,15 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
  * exits.  This call allocates nothing and frees nothing.
  *  - Sizes whose moe_dispatch_workspace_bytes(T, k, E, R) exceeds the
  *    maximum are rejected with MOE_ERR_INVALID_ARG (use moe_dispatch then).
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - The first call in a CUDA context (a device's primary context, or another
+ *    context current at the call) looks up the array's device address there
+ *    with cudaGetSymbolAddress; make that first call before any stream
+ *    capture.  Later calls in the same context reuse the address.  A new
+ *    context (for instance the primary context recreated after
+ *    cudaDeviceReset) has a new id and gets a new lookup, so an address from
+ *    a destroyed context is never reused.
+ *  - A rejected call (MOE_ERR_INVALID_ARG) enqueues nothing and leaves the
+ *    array untouched.
  *  - Every call on a device shares the one array and finds it as the last
  *    call left it; the call clears the part that must start at zero.  Calls
  *    that overlap on the GPU (other streams, other host threads) race on it:
@@ -287,6 +298,37 @@ moe_status moe_combine(const void* y_disp, int dtype, const float* topk_w, const
                        int H, void* y, void* stream);
 
 /*
+ * The masking form of expert parallelism -- [NEURON] "Collective Patterns /
+ * Prefill (CTE kernel)" steps 5-6 and "Why a Single All-Reduce/Reduce-Scatter
+ * Works": every rank runs all tokens against its own experts only, tokens not
+ * routed to them get zeros from it, and a reduce-scatter (prefill) or
+ * all-reduce (decode) sums the ranks' partial outputs.  One GPU holds the R
+ * logical ranks' partials as R planes of one buffer.
+ *
+ * moe_combine_rank_partials: for every rank r and token t,
+ *   y_part[r][t] = sum over j with topk_ids[t][j] / (E / R) == r of
+ *                  topk_w[t][j] * y_disp[slot_to_row[t*k + j]]
+ * (float32, j ascending, rounded once to dtype; zero where rank r owns none
+ * of the token's experts).
+ *   y_disp      [S, H] dtype     expert outputs (moe_expert_ffn)
+ *   topk_w      [T, k] float32, topk_ids [T, k] int32   (moe_route)
+ *   slot_to_row [S] int32        (moe_dispatch; -1 = dropped slot, skipped)
+ *   y_part      [R, T, H] dtype  out
+ * A slot whose row is outside [0, S), or whose id is outside [0, E) with a
+ * row other than -1, contributes nothing and is flagged (bit 4).
+ *
+ * moe_reduce_rank_partials: y[t] = sum over r = 0 .. R-1 of y_part[r][t]
+ * (float32, rank order, rounded once to dtype).
+ *   y_part [R, T, H] dtype, y [T, H] dtype out.
+ * Constraints: H * sizeof(dtype) % 16 == 0; 1 <= k <= 8; E % R == 0,
+ * E <= 1024 (R <= 1024 for the reduction).
+ */
+moe_status moe_combine_rank_partials(const void* y_disp, int dtype, const float* topk_w, const int32_t* topk_ids,
+                                    const int32_t* slot_to_row, int T, int k, int H, int E, int R, void* y_part,
+                                    void* stream);
+moe_status moe_reduce_rank_partials(const void* y_part, int dtype, int T, int H, int R, void* y, void* stream);
+
+/*
  * Expert placement with replicas -- an expert-parallel load balancer:
  * "什么是专家并行（Expert Parallelism）？", "工作机制" and "边界与常见误解"
  * (third point): routing is dynamic, so a balancer redistributes hot and cold
@@ -351,6 +393,25 @@ moe_status moe_get_error(void* stream, uint32_t* bits_out);
  * returns MOE_ERR_TIMEOUT.
  */
 moe_status moe_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+/*
+ * Self-test of moe_dispatch's recovery from a grid-barrier timeout (no
+ * counterpart on the pages: failure detection of this library).  Same
+ * arguments as moe_dispatch (T >= 1), plus limit_us (1 .. 1e6) for each
+ * grid-barrier wait.  It presets the workspace's barrier arrival count to a
+ * value no arrival sequence completes, then launches the dispatch kernel:
+ * every CTA's first barrier wait runs out after limit_us, the timeout bit is
+ * set, the outputs of this call are incomplete, and the kernel's exit
+ * restores the workspace.  A following moe_get_error() returns
+ * MOE_ERR_TIMEOUT, and a following moe_dispatch on the same workspace gives
+ * complete, correct results.
+ */
+moe_status moe_selftest_dispatch_timeout(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k,
+                                         int E, int R, void* x_disp, int32_t* expert_counts,
+                                         int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets,
+                                         int32_t* slot_to_row, int32_t* row_to_slot, int32_t* src_expert_counts,
+                                         void* workspace, size_t workspace_bytes, unsigned int limit_us,
+                                         void* stream);
 
 #ifdef __cplusplus
 }

@@ -76,3 +76,42 @@ class DeviceLayer:
 
 def expert_of_rows(offsets: np.ndarray, rows: np.ndarray) -> np.ndarray:
     return (np.searchsorted(offsets, rows, side="right") - 1).astype(np.int32)
+
+
+def row_errors(gpu: np.ndarray, ref: np.ndarray) -> tuple[float, float, int]:
+    """(normwise error of the whole tensor, worst per-row normwise error, that row's index):
+    the per-row figure scales each row by its own largest reference value, so one wrong tile
+    cannot hide under the tensor-wide maximum."""
+    ref = np.asarray(ref, np.float64)
+    g = widen(gpu) if gpu.dtype == np.uint16 else gpu.astype(np.float64)
+    diff = np.abs(g - ref)
+    whole = float(diff.max() / max(np.abs(ref).max(), 1e-300)) if ref.size else 0.0
+    if not ref.size:
+        return whole, 0.0, -1
+    per_row = diff.max(axis=1) / np.maximum(np.abs(ref).max(axis=1), 1e-300)
+    worst = int(np.argmax(per_row))
+    return whole, float(per_row[worst]), worst
+
+
+def oracle_ffn_rows_by_expert(layer: "DeviceLayer", rows: np.ndarray, row_to_slot: np.ndarray,
+                              expert_offsets: np.ndarray, host_bytes: int = 2 << 30):
+    """The oracle's SwiGLU outputs (h, y_disp) of the given dispatched rows, in float64.
+
+    Each row's input is its token's row of x (the oracle's dispatch: x_disp[r] = x[row_to_slot[r] / k]);
+    the experts' weights are regenerated on the host a few experts at a time (at most
+    ``host_bytes`` of weights at once), so the largest layers fit."""
+    wl = layer.wl
+    rows = np.asarray(rows, np.int64)
+    experts = expert_of_rows(expert_offsets, rows)
+    x_rows = layer.x[row_to_slot[rows] // wl.k]
+    h = np.empty((len(rows), wl.I), np.float64)
+    y = np.empty((len(rows), wl.H), np.float64)
+    per_expert = 3 * wl.H * wl.I * (2 if wl.dtype == "bf16" else 4)
+    step = max(1, host_bytes // per_expert)
+    uniq = np.unique(experts)
+    for i in range(0, len(uniq), step):
+        es = uniq[i:i + step]
+        sel = np.isin(experts, es)
+        g, u, d = layer.host_weights(es)
+        y[sel], h[sel] = oracle.ffn_rows(x_rows[sel], experts[sel], g, u, d, wl.H, wl.I, want_act=True)
+    return h, y

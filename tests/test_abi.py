@@ -89,6 +89,31 @@ def test_dispatch_rejects(kw, needle):
     assert needle in _native.lib().moe_last_error_message()
 
 
+def test_noalloc_dispatch_rejects_bad_arguments_before_any_device_work():
+    """Sizes within the built-in scratch but a bad argument: rejected on the host by the same
+    checks as moe_dispatch (no CUDA call is made, so this runs without a GPU)."""
+    lib = _native.lib()
+    args = [FAKE, 1, 8, 64, FAKE, 2, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None]
+    bad = list(args)
+    bad[7] = 3  # R does not divide E
+    assert lib.moe_dispatch_noalloc(*bad, None) == _native.MOE_ERR_INVALID_ARG
+    assert b"divide E" in lib.moe_last_error_message()
+    bad = list(args)
+    bad[13] = None  # slot_to_row
+    assert lib.moe_dispatch_noalloc(*bad, None) == _native.MOE_ERR_INVALID_ARG
+    assert b"slot_to_row" in lib.moe_last_error_message()
+
+
+@pytest.mark.parametrize("limit_us,T,needle", [(0, 8, b"limit_us"), (2000000, 8, b"limit_us"), (20, 0, b"T must"),
+                                               (20, -3, b"T must")])
+def test_dispatch_timeout_selftest_rejects(limit_us, T, needle):
+    lib = _native.lib()
+    st = lib.moe_selftest_dispatch_timeout(FAKE, 1, T, 64, FAKE, 2, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                           None, FAKE, 1 << 20, limit_us, None)
+    assert st == _native.MOE_ERR_INVALID_ARG
+    assert needle in lib.moe_last_error_message()
+
+
 @pytest.mark.parametrize("kw,needle", [
     (dict(k=9), b"k must"),
     (dict(S=17), b"S must be <= T * k"),

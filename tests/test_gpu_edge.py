@@ -178,3 +178,44 @@ def test_dispatch_index_against_oracle(T, E, k, R):
             assert (dev_to_np(getattr(out, key)) == ref[key]).all(), key
         xd = oracle.dispatch_rows(dev_to_np(x), k, ref["slot_to_row"])
         assert (dev_to_np(out.x_disp) == xd).all()
+
+
+@pytest.mark.parametrize("T,E,k,R,index_only", [(512, 8, 2, 4, False),     # one grid barrier (count table in smem)
+                                                (2048, 1024, 8, 32, False),  # two grid barriers
+                                                (777, 64, 4, 8, True)])     # index-only dispatch
+def test_dispatch_recovers_from_grid_barrier_timeout(T, E, k, R, index_only):
+    """A dispatch whose grid barrier times out reports MOE_ERR_TIMEOUT, and the next
+    moe_dispatch on the same workspace is complete and exact: the kernel's last CTA
+    to finish zeroes the barrier's counters on every exit path."""
+    m = _api()
+    from token_dispatch_combine_b200 import _native
+    lib = _native.lib()
+    rng = np.random.default_rng(T + k)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    ids, _ = oracle.route(logits, k)
+    ids_dev = torch.from_numpy(ids).cuda()
+    H = 64
+    x = torch.randn(T, H, device="cuda").to(torch.bfloat16)
+    out = m.DispatchOut.empty(T, H, k, E, R, torch.bfloat16, "cuda", rows=not index_only)
+    ws = m.new_dispatch_workspace(T, k, E, R, "cuda")
+    xp = None if index_only else x.data_ptr()
+    xdp = None if index_only else out.x_disp.data_ptr()
+    args = [xp, _native.MOE_BF16, T, H, ids_dev.data_ptr(), k, E, R, xdp, out.expert_counts.data_ptr(),
+            out.expert_offsets.data_ptr(), out.rank_counts.data_ptr(), out.rank_offsets.data_ptr(),
+            out.slot_to_row.data_ptr(), out.row_to_slot.data_ptr(), out.src_expert_counts.data_ptr(),
+            ws.data_ptr(), ws.numel()]
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.moe_selftest_dispatch_timeout(*args, 20, stream) == 0  # 20 us per barrier wait
+    st, bits = m.moe_get_error()
+    assert st == _native.MOE_ERR_TIMEOUT and bits & _native.ERR_TIMEOUT
+    ctrl = ws[:256].view(torch.int32).cpu()
+    assert int(ctrl[16]) == 0 and int(ctrl[48]) == 0  # arrival count (byte 64), exit count (byte 192)
+    for _ in range(2):
+        m.moe_dispatch(None if index_only else x, ids_dev, E, R, out, ws, H=H, dtype=torch.bfloat16)
+        assert m.moe_get_error() == (0, 0)
+        ref = oracle.dispatch_index(ids, E, R)
+        for key in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "slot_to_row", "row_to_slot",
+                    "src_expert_counts"):
+            assert (dev_to_np(getattr(out, key)) == ref[key]).all(), key
+        if not index_only:
+            assert (dev_to_np(out.x_disp) == oracle.dispatch_rows(dev_to_np(x), k, ref["slot_to_row"])).all()

@@ -25,6 +25,7 @@ EXPORTS = (
     "moe_dispatch", "moe_expert_ffn", "moe_ffn_gate_up", "moe_ffn_down", "moe_combine", "moe_get_error", "moe_selftest_wait_timeout",
     "moe_dispatch_noalloc", "moe_set_ffn_tiling", "moe_get_ffn_tiling", "moe_ffn_tiling_for", "moe_router_topk",
     "moe_ffn_gate_up_gather", "moe_expert_ffn_gather", "moe_eplb_plan", "moe_eplb_remap", "moe_eplb_replicate",
+    "moe_selftest_dispatch_timeout", "moe_combine_rank_partials", "moe_reduce_rank_partials",
 )
 
 _lock = threading.Lock()
@@ -62,6 +63,10 @@ def _configure(lib):
         "moe_eplb_plan": ([vp, i32, i32, i32, vp, vp, vp], i32),
         "moe_eplb_remap": ([vp, i32, i32, i32, vp, vp, i32, vp, vp], i32),
         "moe_eplb_replicate": ([vp, sz, i32, vp, i32, vp, vp], i32),
+        "moe_combine_rank_partials": ([vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp], i32),
+        "moe_reduce_rank_partials": ([vp, i32, i32, i32, i32, vp, vp], i32),
+        "moe_selftest_dispatch_timeout": ([vp, i32, i32, i32, vp, i32, i32, i32] + [vp] * 8 + [vp, sz, ctypes.c_uint, vp],
+                                          i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)

@@ -30,8 +30,11 @@
 //     the counting and the barriers.
 // With x_disp == nullptr (index-only dispatch, for a gate/up GEMM that gathers
 // its rows from x itself) phase 3 writes only the permutation.
-// A barrier that does not complete within 1 s sets the timeout bit of the
-// device error word; the kernel then returns without writing the rows.
+// A barrier that does not complete within its limit (1 s for moe_dispatch)
+// sets the timeout bit of the device error word; the CTA then skips the rest
+// of its work.  Every CTA, on every path, ends by arriving on an exit counter,
+// and the last one out zeroes the barrier's arrival counter and the exit
+// counter: a call that timed out leaves the workspace ready for the next one.
 #pragma once
 
 #include "common.cuh"
@@ -43,7 +46,7 @@ constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kScatterVecsPerLane = 4;                   // 16-byte vectors in flight per lane
 constexpr int kScatterSlice = 32 * kScatterVecsPerLane;  // 16-byte vectors of a row per warp item
 constexpr int kRowRound = kDispatchThreads / 8;          // tokens per phase-3 round: one slot per thread at k <= 8
-constexpr uint64_t kGridBarrierLimitNs = 1000000000ull;   // 1 s
+constexpr uint64_t kGridBarrierLimitNs = 1000000000ull;   // 1 s: the limit of every moe_dispatch call
 // Count tables up to this many entries are scanned by every CTA in shared
 // memory, which saves the second grid barrier.
 constexpr size_t kSmallCountTable = 8192;
@@ -85,11 +88,15 @@ inline DispatchGeom make_dispatch_geom(int T, int k, int E, int R) {
 }
 
 // Workspace layout (bytes): [0,256) control words (grid-barrier arrival count
-// at 64, generation at 128); chunk_counts[nchunks][E]; chunk_base[nchunks][E]
-// (relative to the expert's offset); slot_rank[S]; totals[E].
+// at 64, generation at 128, exit count at 192; the two counts are zero
+// between calls, the generation takes any value); chunk_counts[nchunks][E];
+// chunk_base[nchunks][E] (relative to the expert's offset); slot_rank[S];
+// totals[E].
+constexpr size_t kDispatchBarCountOffset = 64;
 struct DispatchWs {
   uint32_t* bar_count;
   uint32_t* bar_gen;
+  uint32_t* exit_count;
   int32_t* chunk_counts;
   int32_t* chunk_base;
   int32_t* slot_rank;
@@ -103,8 +110,9 @@ inline size_t dispatch_ws_bytes(const DispatchGeom& g) {
 inline DispatchWs dispatch_ws_carve(void* base, const DispatchGeom& g) {
   char* p = (char*)base;
   DispatchWs w;
-  w.bar_count = (uint32_t*)(p + 64);
+  w.bar_count = (uint32_t*)(p + kDispatchBarCountOffset);
   w.bar_gen = (uint32_t*)(p + 128);
+  w.exit_count = (uint32_t*)(p + 192);
   w.chunk_counts = (int32_t*)(p + 256);
   w.chunk_base = w.chunk_counts + (size_t)g.nchunks * g.E;
   w.slot_rank = w.chunk_base + (size_t)g.nchunks * g.E;
@@ -136,9 +144,9 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 
 // Grid-wide barrier for a cooperative launch.  Thread 0 of each CTA reads the
 // generation, arrives on the counter; the last arrival resets the counter and
-// bumps the generation; the others wait (bounded) for the bump.  Returns
-// false, with the timeout bit set, if the wait gave up.
-__device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok) {
+// bumps the generation; the others wait (at most limit_ns) for the bump.
+// Returns false, with the timeout bit set, if the wait gave up.
+__device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok, uint64_t limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint32_t gen = ld_acquire_u32(ws.bar_gen);
@@ -151,7 +159,7 @@ __device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok) {
     } else {
       const uint64_t t0 = globaltimer_ns();
       while (ld_acquire_u32(ws.bar_gen) == gen) {
-        if (globaltimer_ns() - t0 > kGridBarrierLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
           flag_error(kErrTimeout);
           *s_ok = 0;
           break;
@@ -165,15 +173,29 @@ __device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok) {
   return *s_ok != 0;
 }
 
+// Last step of every CTA on every path (thread 0 only, after its last barrier
+// operation): arrive on the exit counter; the last CTA out zeroes the arrival
+// and exit counters.  A barrier that timed out leaves a partial arrival count
+// behind, so without this the next call on the workspace would start from it.
+__device__ __forceinline__ void dispatch_exit(const DispatchWs& ws) {
+  if (threadIdx.x != 0) return;
+  __threadfence();
+  if (atomicAdd(ws.exit_count, 1u) == gridDim.x - 1) {
+    atomicExch(ws.bar_count, 0u);
+    atomicExch(ws.exit_count, 0u);
+    __threadfence();
+  }
+}
+
 // Dynamic shared memory: warp_counts[kDispatchWarps][E] int32 (or the whole
 // [nchunks][E] table when it is small and larger), then offs[E + 1], then the
 // rows of one round of this CTA's slots, rows[kDispatchThreads].
 template <typename T>
-__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
-    DispatchGeom g, int H, int nslices, int tpc, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
-    T* __restrict__ x_disp, int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
-    int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_to_row,
-    int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
+__device__ __forceinline__ void dispatch_phases(
+    const DispatchGeom& g, int H, int nslices, int tpc, const T* __restrict__ x, const int32_t* __restrict__ ids,
+    const DispatchWs& ws, uint64_t limit_ns, T* __restrict__ x_disp, int32_t* __restrict__ expert_counts,
+    int32_t* __restrict__ expert_offsets, int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets,
+    int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
   extern __shared__ int32_t smem_i32[];
   int32_t* warp_counts = smem_i32;                                    // [kDispatchWarps][E]
   int32_t* offs = smem_i32 + dispatch_smem_table(g.nchunks, g.E);     // [E + 1]
@@ -249,7 +271,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
     if (s < s1) ws.slot_rank[s] = (e >= 0) ? warp_counts[warp * g.E + e] + rank_in_warp : -1;
     __syncthreads();  // warp_counts is reused by the next chunk
   }
-  if (!grid_barrier(ws, &s_ok)) return;
+  if (!grid_barrier(ws, &s_ok, limit_ns)) return;
 
   if (small_table) {
     // ---- phase 2 (small count table): every CTA scans the whole table itself
@@ -286,7 +308,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
       expert_counts[e] = carry;
     }
   }
-  if (!grid_barrier(ws, &s_ok)) return;
+  if (!grid_barrier(ws, &s_ok, limit_ns)) return;
 
   // ---- phase 2b: expert offsets (every CTA, in shared memory)
   for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) offs[xx] = __ldcg(ws.totals + xx);
@@ -391,10 +413,22 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
 }
 
 template <typename T>
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
+    DispatchGeom g, int H, int nslices, int tpc, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
+    uint64_t limit_ns, T* __restrict__ x_disp, int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
+    int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_to_row,
+    int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
+  dispatch_phases<T>(g, H, nslices, tpc, x, ids, ws, limit_ns, x_disp, expert_counts, expert_offsets, rank_counts,
+                     rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
+  dispatch_exit(ws);
+}
+
+// limit_ns bounds each grid-barrier wait (kGridBarrierLimitNs for moe_dispatch).
+template <typename T>
 cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int32_t* ids, void* workspace,
                             T* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
                             int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
-                            int32_t* src_expert_counts, cudaStream_t stream) {
+                            int32_t* src_expert_counts, cudaStream_t stream, uint64_t limit_ns = kGridBarrierLimitNs) {
   DispatchWs ws = dispatch_ws_carve(workspace, g);
   auto kern = dispatch_kernel<T>;
   const size_t smem = sizeof(int32_t) * (dispatch_smem_table(g.nchunks, g.E) + g.E + 1 + kDispatchThreads);
@@ -438,8 +472,8 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = MOE_PDL ? 2 : 1;
-  err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, tpc, x, ids, ws, x_disp, expert_counts, expert_offsets, rank_counts,
-                           rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
+  err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, tpc, x, ids, ws, limit_ns, x_disp, expert_counts, expert_offsets,
+                           rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

@@ -3,6 +3,8 @@
 // Host side only validates arguments, picks kernel configurations and
 // enqueues launches on the caller's stream.  It never allocates, never copies
 // to the host and never synchronises (moe_get_error excepted).
+#include <cuda.h>
+
 #include <atomic>
 #include <cstdio>
 #include <mutex>
@@ -16,6 +18,7 @@
 #include "ffn_tc2.cuh"
 #include "route.cuh"
 #include "eplb.cuh"
+#include "masked.cuh"
 #include "router.cuh"
 
 namespace {
@@ -148,10 +151,18 @@ size_t moe_dispatch_workspace_bytes(int T, int k, int E, int R) {
   return moe::dispatch_ws_bytes(moe::make_dispatch_geom(T, k, E, R));
 }
 
-moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
-                        void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
-                        int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
-                        int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Host-side checks of a dispatch call; nothing is enqueued.  The workspace
+// pointer and size are checked only when `check_workspace` is set (the
+// no-alloc form supplies its own).
+moe_status check_dispatch(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
+                          const void* x_disp, const int32_t* expert_counts, const int32_t* expert_offsets,
+                          const int32_t* rank_counts, const int32_t* rank_offsets, const int32_t* slot_to_row,
+                          const int32_t* row_to_slot, const int32_t* src_expert_counts, bool check_workspace,
+                          const void* workspace, size_t workspace_bytes) {
   const size_t es = dtype_size(dtype);
   MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
   MOE_REQUIRE(T >= 0, "T must be >= 0");
@@ -165,9 +176,11 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
   MOE_REQUIRE_PTR(rank_counts, 4, "rank_counts");
   MOE_REQUIRE_PTR(rank_offsets, 4, "rank_offsets");
   MOE_REQUIRE(src_expert_counts == nullptr || aligned(src_expert_counts, 4), "src_expert_counts misaligned");
-  MOE_REQUIRE_PTR(workspace, 16, "workspace");
-  const moe::DispatchGeom g = moe::make_dispatch_geom(T, k, E, R);
-  MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(g), "workspace_bytes smaller than moe_dispatch_workspace_bytes()");
+  if (check_workspace) {
+    MOE_REQUIRE_PTR(workspace, 16, "workspace");
+    MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(moe::make_dispatch_geom(T, k, E, R)),
+                "workspace_bytes smaller than moe_dispatch_workspace_bytes()");
+  }
   MOE_REQUIRE((x == nullptr) == (x_disp == nullptr),
               "x and x_disp must both be given, or both be NULL (index-only dispatch)");
   if (T > 0) {
@@ -179,17 +192,64 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
     MOE_REQUIRE_PTR(slot_to_row, 4, "slot_to_row");
     MOE_REQUIRE_PTR(row_to_slot, 4, "row_to_slot");
   }
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t err;
+  return MOE_OK;
+}
+
+// Enqueues the dispatch kernel of a call that passed check_dispatch.
+cudaError_t enqueue_dispatch(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
+                             void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                             int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
+                             int32_t* src_expert_counts, void* workspace, cudaStream_t s,
+                             uint64_t limit_ns = moe::kGridBarrierLimitNs) {
+  const moe::DispatchGeom g = moe::make_dispatch_geom(T, k, E, R);
   if (dtype == MOE_BF16)
-    err = moe::launch_dispatch(g, H, (const __nv_bfloat16*)x, topk_ids, workspace, (__nv_bfloat16*)x_disp,
-                               expert_counts, expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
-                               src_expert_counts, s);
-  else
-    err = moe::launch_dispatch(g, H, (const float*)x, topk_ids, workspace, (float*)x_disp, expert_counts,
-                               expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
-                               src_expert_counts, s);
-  return cuda_status(err, "moe_dispatch");
+    return moe::launch_dispatch(g, H, (const __nv_bfloat16*)x, topk_ids, workspace, (__nv_bfloat16*)x_disp,
+                                expert_counts, expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
+                                src_expert_counts, s, limit_ns);
+  return moe::launch_dispatch(g, H, (const float*)x, topk_ids, workspace, (float*)x_disp, expert_counts,
+                              expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts,
+                              s, limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
+                        void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                        int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
+                        int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream) {
+  moe_status st = check_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                 rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts, true,
+                                 workspace, workspace_bytes);
+  if (st != MOE_OK) return st;
+  return cuda_status(enqueue_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                      rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts,
+                                      workspace, (cudaStream_t)stream),
+                     "moe_dispatch");
+}
+
+moe_status moe_selftest_dispatch_timeout(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k,
+                                         int E, int R, void* x_disp, int32_t* expert_counts,
+                                         int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets,
+                                         int32_t* slot_to_row, int32_t* row_to_slot, int32_t* src_expert_counts,
+                                         void* workspace, size_t workspace_bytes, unsigned int limit_us,
+                                         void* stream) {
+  MOE_REQUIRE(limit_us >= 1 && limit_us <= 1000000u, "limit_us must be in [1, 1000000]");
+  MOE_REQUIRE(T >= 1, "T must be >= 1 (a call with no tokens launches nothing)");
+  moe_status st = check_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                 rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts, true,
+                                 workspace, workspace_bytes);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  // An arrival count far above any grid size: no arrival can be the last, so
+  // the first grid barrier runs out in every CTA.
+  cudaError_t err = cudaMemsetAsync(static_cast<char*>(workspace) + moe::kDispatchBarCountOffset, 0x40, 4, s);
+  if (err != cudaSuccess) return cuda_status(err, "moe_selftest_dispatch_timeout: preset arrival count");
+  return cuda_status(enqueue_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                      rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts,
+                                      workspace, s, (uint64_t)limit_us * 1000ull),
+                     "moe_selftest_dispatch_timeout");
 }
 
 // ---------------------------------------------------------------------------
@@ -202,29 +262,79 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
 // them the dispatch scratch lives in the array below, which the CUDA module
 // reserves on every GPU that loads this library and keeps until the process
 // exits.  Host code never touches the array by name (that name is only a
-// host-side stand-in); its device address is looked up once per device with
-// cudaGetSymbolAddress and passed to the kernels.
+// host-side stand-in); its device address is looked up with
+// cudaGetSymbolAddress once per CUDA context (the device's primary context,
+// or any other context current at the call) and passed to the kernels.
 static __device__ __align__(256) unsigned char g_dispatch_noalloc_scratch[MOE_DISPATCH_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kNoallocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kNoallocMaxDevices] = {};
+// cuCtxGetCurrent / cuCtxGetId, fetched from the driver through the runtime
+// (no link against libcuda).  Context ids are unique for the life of the
+// process, so a context created later (after cudaDeviceReset, or one a caller
+// made current with the driver API) never matches an old entry.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device (looked up on the first call there).
+struct NoallocEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+constexpr int kNoallocEntries = 64;
+std::mutex g_noalloc_mu;
+NoallocEntry g_noalloc_cache[kNoallocEntries] = {};
+int g_noalloc_next = 0;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+moe_status current_context_id(unsigned long long* id) {
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) {
+    void* f0 = nullptr;
+    void* f1 = nullptr;
+    cudaDriverEntryPointQueryResult q0, q1;
+    cudaError_t err = cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f0, 12000, cudaEnableDefault, &q0);
+    if (err == cudaSuccess)
+      err = cudaGetDriverEntryPointByVersion("cuCtxGetId", &f1, 12000, cudaEnableDefault, &q1);
+    if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: driver entry points");
+    if (q0 != cudaDriverEntryPointSuccess || q1 != cudaDriverEntryPointSuccess || !f0 || !f1)
+      return fail(MOE_ERR_CUDA, "moe_dispatch_noalloc: cuCtxGetCurrent/cuCtxGetId not available");
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f0);
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f1);
+  }
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || g_ctx_get_id(ctx, id) != CUDA_SUCCESS)
+    return fail(MOE_ERR_CUDA, "moe_dispatch_noalloc: no current CUDA context");
+  return MOE_OK;
+}
+
+// Device address of the scratch array in the current context: looked up with
+// cudaGetSymbolAddress on the first call in a context (the set-up step), then
+// taken from the table.
 moe_status noalloc_scratch(void** out) {
   int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  cudaError_t err = cudaGetDevice(&dev);  // the runtime makes the device's primary context current if none is
   if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: cudaGetDevice");
-  if (dev < 0 || dev >= kNoallocMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "moe_dispatch_noalloc: device index too large");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  unsigned long long id = 0;
+  moe_status st = current_context_id(&id);
+  if (st != MOE_OK) {
+    // A context the runtime has not created yet: the symbol lookup creates it.
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_dispatch_noalloc_scratch);
     if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: cudaGetSymbolAddress");
-    g_noalloc_addr[dev] = p;
+    st = current_context_id(&id);
+    if (st != MOE_OK) return st;
   }
-  *out = g_noalloc_addr[dev];
+  for (const NoallocEntry& e : g_noalloc_cache)
+    if (e.addr != nullptr && e.ctx_id == id) {
+      *out = e.addr;
+      return MOE_OK;
+    }
+  void* p = nullptr;
+  err = cudaGetSymbolAddress(&p, g_dispatch_noalloc_scratch);
+  if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: cudaGetSymbolAddress");
+  g_noalloc_cache[g_noalloc_next] = NoallocEntry{id, p};
+  g_noalloc_next = (g_noalloc_next + 1) % kNoallocEntries;
+  *out = p;
   return MOE_OK;
 }
 }  // namespace
@@ -234,6 +344,8 @@ extern "C" moe_status moe_dispatch_noalloc(const void* x, int dtype, int T, int 
                                            int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets,
                                            int32_t* slot_to_row, int32_t* row_to_slot, int32_t* src_expert_counts,
                                            void* stream) {
+  // 1. sizes against the built-in scratch, 2. every other argument, 3. only
+  // then any device work: a rejected call enqueues nothing.
   MOE_REQUIRE(T >= 0 && k >= 1 && E >= 1 && R >= 1, "T >= 0, k >= 1, E >= 1 and R >= 1 are required");
   MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
   const size_t need = moe_dispatch_workspace_bytes(T, k, E, R);
@@ -241,15 +353,21 @@ extern "C" moe_status moe_dispatch_noalloc(const void* x, int dtype, int T, int 
               "moe_dispatch_noalloc: these sizes need " + std::to_string(need) +
                   " bytes of scratch, more than the built-in " +
                   std::to_string((size_t)MOE_DISPATCH_NOALLOC_SCRATCH_BYTES) + "; use moe_dispatch with a workspace");
-  void* scratch = nullptr;
-  moe_status st = noalloc_scratch(&scratch);
+  moe_status st = check_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                 rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts, false,
+                                 nullptr, 0);
   if (st != MOE_OK) return st;
-  // The array keeps whatever the previous call left; the control word must start at zero.
-  cudaError_t err = cudaMemsetAsync(scratch, 0, 256, (cudaStream_t)stream);
-  if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: clear control word");
-  return moe_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets, rank_counts,
-                      rank_offsets, slot_to_row, row_to_slot, src_expert_counts, scratch,
-                      (size_t)MOE_DISPATCH_NOALLOC_SCRATCH_BYTES, stream);
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  // The array keeps whatever the previous call left; the control words must start at zero.
+  cudaError_t err = cudaMemsetAsync(scratch, 0, 256, s);
+  if (err != cudaSuccess) return cuda_status(err, "moe_dispatch_noalloc: clear control words");
+  return cuda_status(enqueue_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                      rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts, scratch,
+                                      s),
+                     "moe_dispatch_noalloc");
 }
 
 static moe_status check_ffn(int dtype, int E, int H, int I, int S, const void* a, const char* a_name,
@@ -369,6 +487,52 @@ moe_status moe_combine(const void* y_disp, int dtype, const float* topk_w, const
   else
     err = moe::launch_combine((const float*)y_disp, topk_w, slot_to_row, T, k, H, (float*)y, s);
   return cuda_status(err, "moe_combine");
+}
+
+moe_status moe_combine_rank_partials(const void* y_disp, int dtype, const float* topk_w, const int32_t* topk_ids,
+                                    const int32_t* slot_to_row, int T, int k, int H, int E, int R, void* y_part,
+                                    void* stream) {
+  const size_t es = dtype_size(dtype);
+  MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  MOE_REQUIRE(k >= 1 && k <= 8, "k must be in [1, 8]");
+  MOE_REQUIRE(H >= 1 && (H * es) % 16 == 0, "H * sizeof(dtype) must be a positive multiple of 16");
+  MOE_REQUIRE(E >= 1 && E <= 1024, "E must be in [1, 1024]");
+  MOE_REQUIRE(R >= 1 && E % R == 0, "R must be >= 1 and divide E");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(y_disp, 16, "y_disp");
+  MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
+  MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
+  MOE_REQUIRE_PTR(slot_to_row, 4, "slot_to_row");
+  MOE_REQUIRE_PTR(y_part, 16, "y_part");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = moe::launch_rank_partials((const __nv_bfloat16*)y_disp, topk_w, topk_ids, slot_to_row, T, k, H, E, R,
+                                    (__nv_bfloat16*)y_part, s);
+  else
+    err = moe::launch_rank_partials((const float*)y_disp, topk_w, topk_ids, slot_to_row, T, k, H, E, R,
+                                    (float*)y_part, s);
+  return cuda_status(err, "moe_combine_rank_partials");
+}
+
+moe_status moe_reduce_rank_partials(const void* y_part, int dtype, int T, int H, int R, void* y, void* stream) {
+  const size_t es = dtype_size(dtype);
+  MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  MOE_REQUIRE(H >= 1 && (H * es) % 16 == 0, "H * sizeof(dtype) must be a positive multiple of 16");
+  MOE_REQUIRE(R >= 1 && R <= 1024, "R must be in [1, 1024]");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(y_part, 16, "y_part");
+  MOE_REQUIRE_PTR(y, 16, "y");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = moe::launch_reduce_ranks((const __nv_bfloat16*)y_part, T, H, R, (__nv_bfloat16*)y, s);
+  else
+    err = moe::launch_reduce_ranks((const float*)y_part, T, H, R, (float*)y, s);
+  return cuda_status(err, "moe_reduce_rank_partials");
 }
 
 moe_status moe_eplb_plan(const int64_t* load, int E, int R, int slots_per_rank, int32_t* phys_to_logical,
