@@ -281,8 +281,10 @@ def run_ours(args, wl):
 
     x, logits = up(x_np), up(logits_np)
     wg, wu, wd = up(wg_np), up(wu_np), up(wd_np)
+    rc = args.route_counts == "on"
     rt = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev,
-                      gather={"auto": "auto", "rows": False, "gather": True}[args.dispatch])
+                      gather={"auto": "auto", "rows": False, "gather": True}[args.dispatch], route_counts=rc,
+                      combine_in_down=args.combine_in_down == "on")
     gather = rt.gather
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     flush_max = torch.empty((), dtype=torch.int32, device=dev)
@@ -355,8 +357,8 @@ def run_ours(args, wl):
     # The dispatch+combine metric is about the row-moving dispatch: when the step gathers its
     # rows in the gate/up projection, measure dispatch (with rows) and combine on a second,
     # row-moving round trip of the same layer.
-    if gather:
-        rt_dc = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev, gather=False)
+    if gather or rt.combine_in_down:  # (the metric's combine is moe_combine on y_disp)
+        rt_dc = MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev, gather=False, route_counts=rc)
         rt_dc.forward(x, logits, wg, wu, wd)
         dc_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
         for ev in dc_ev:
@@ -389,7 +391,8 @@ def run_ours(args, wl):
     # Dispatch + combine as a stream of layers: 4 independent buffer sets (x, dispatched rows,
     # y_disp, y: ~1.3 GB, far beyond the 126 MB L2) visited in turn, 20 pairs under one event pair.
     # Launch latency is then overlapped as it is inside a step, and no pair finds its data in L2.
-    sets = [MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev, gather=False) for _ in range(4)]
+    sets = [MoERoundTrip(wl.T, wl.H, wl.I, wl.E, wl.k, wl.R, dt, device=dev, gather=False, route_counts=rc)
+            for _ in range(4)]
     xs = [x.clone() for _ in sets]
     for r_, x_ in zip(sets, xs):
         r_.route(logits)
@@ -406,8 +409,43 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     dc_stream_ms = a.elapsed_time(b) / n_pairs
     del sets, xs
-    if gather:
+    if rt_dc is not rt:
         del rt_dc
+
+    # The masking form's return path (moe_combine_rank_partials + moe_reduce_rank_partials) in
+    # place of combine, on this step's y_disp: R per-rank partial planes, then their rank-ordered
+    # sum; L2 flushed before each kernel.
+    masked = None
+    if wl.R > 1:
+        from token_dispatch_combine_b200 import moe_combine_rank_partials, moe_reduce_rank_partials
+        y_part = torch.empty((wl.R, wl.T, wl.H), dtype=dt, device=dev)
+        y_m = torch.empty((wl.T, wl.H), dtype=dt, device=dev)
+        mev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        for ev in mev:
+            flush_and_hold()
+            ev[0].record(stream)
+            moe_combine_rank_partials(rt.y_disp, rt.topk_w, rt.topk_ids, rt.disp.slot_to_row, wl.E, wl.R, y_part)
+            ev[1].record(stream)
+            flush_and_hold()
+            ev[2].record(stream)
+            moe_reduce_rank_partials(y_part, y_m)
+            ev[3].record(stream)
+        torch.cuda.synchronize()
+        st, bits = moe_get_error()
+        if st != 0:
+            raise RuntimeError(f"device error word {bits} in the masking form")
+        b_ = 2 if wl.dtype == "bf16" else 4
+        part_us = statistics.median(ev[0].elapsed_time(ev[1]) for ev in mev) * 1e3
+        red_us = statistics.median(ev[2].elapsed_time(ev[3]) for ev in mev) * 1e3
+        part_bytes = wl.S * wl.H * b_ + wl.R * wl.T * wl.H * b_ + 12 * wl.S
+        red_bytes = wl.R * wl.T * wl.H * b_ + wl.T * wl.H * b_
+        masked = {"rank_partials_us": part_us, "reduce_us": red_us,
+                  "rank_partials_gbs": part_bytes / (part_us * 1e-6) / 1e9,
+                  "reduce_gbs": red_bytes / (red_us * 1e-6) / 1e9,
+                  "extra_us_vs_combine": part_us + red_us - float(stage[4]) * 1e3,
+                  "bytes": "partials S*H*b + R*T*H*b + 12*S; reduction R*T*H*b + T*H*b",
+                  "timing": "events per kernel, L2 flushed before each, median of the steps"}
+        del y_part, y_m
 
     # The router affinities fused with the top-k (moe_router_topk): logits = x W_r^T + bias on
     # tensor cores, then route's selection; L2 flushed before each call.  Not part of the step
@@ -533,6 +571,10 @@ def run_ours(args, wl):
     t_route, t_disp, t_gu, t_down, t_comb = stage_max
     gemm_tflops = (alg["gateup_flops"] + alg["down_flops"]) / ((t_gu + t_down) * 1e-3) / 1e12
     dc_gbs = (alg["dispatch_bytes"] + alg["combine_bytes"]) / ((t_disp_rows + t_comb_rows) * 1e-3) / 1e9
+    # the same with the routing kernel's time and bytes included (it holds the dispatch's counting
+    # when route_counts is on)
+    rdc_gbs = (alg["route_bytes"] + alg["dispatch_bytes"] + alg["combine_bytes"]) / (
+        (t_route + t_disp_rows + t_comb_rows) * 1e-3) / 1e9
     gu_tflops = alg["gateup_flops"] / (t_gu * 1e-3) / 1e12
     peak_tf = peaks["bf16_tflops"]
     tiling = moe_ffn_tiling_for(wl.E, wl.S, FFN_GATE_UP)
@@ -572,6 +614,11 @@ def run_ours(args, wl):
             "route_us": t_route * 1e3, "dispatch_us": t_disp * 1e3, "gate_up_us": t_gu * 1e3,
             "down_us": t_down * 1e3, "combine_us": t_comb * 1e3,
             "dispatch_rows_us": t_disp_rows * 1e3,
+            "combine": ("in the down projection's epilogue (moe_ffn_down_combine) + finalize"
+                        if rt.combine_in_down else "moe_combine"),
+            "dispatch_counting": ("in the routing kernel (moe_route_count; the dispatch kernel scans the chunk "
+                                  "counts, permutes and copies)" if rc else "in the dispatch kernel (moe_dispatch)"),
+            "route_dispatch_combine_gbs": rdc_gbs, "route_dispatch_combine_frac_hbm": rdc_gbs / peaks["hbm_gbs"],
             "dispatch_combine_gbs": dc_gbs, "dispatch_combine_frac_hbm": dc_gbs / peaks["hbm_gbs"],
             "dispatch_combine_back_to_back_us": dc_pair_ms * 1e3,
             "dispatch_combine_back_to_back_gbs": (alg["dispatch_bytes"] + alg["combine_bytes"]) / (dc_pair_ms * 1e-3) / 1e9,
@@ -595,6 +642,7 @@ def run_ours(args, wl):
                 "router_topk_timing": "moe_router_topk (logits = x W_r^T + bias, then top-k), L2 flushed, "
                                       "events per call; bytes T*H*2 + E*H*2 + T*k*8"}),
             **({} if eplb is None else {"eplb": eplb}),
+            **({} if masked is None else {"masking_form": masked}),
             "graph_replay_ms": graph_ms,
             **({} if graph_err is None else {"graph_replay_error": graph_err}),
             "ffn_tiling": {"gate_up": "pair" if tiling == FFN_TILING_PAIR else "single",
@@ -635,6 +683,12 @@ def main():
     ap.add_argument("--dispatch", default="auto", choices=["auto", "rows", "gather"],
                     help="rows: dispatch writes x_disp; gather: index-only dispatch, the gate/up projection "
                          "gathers its rows from x (moe_ffn_gate_up_gather); auto: MoERoundTrip's choice")
+    ap.add_argument("--route-counts", default="on", choices=["on", "off"],
+                    help="on: the routing kernel also does the dispatch's counting (moe_route_count + "
+                         "moe_dispatch_counted); off: moe_route + moe_dispatch")
+    ap.add_argument("--combine-in-down", default="off", choices=["on", "off"],
+                    help="on: the down projection's epilogue does the combine (moe_ffn_down_combine, float32 "
+                         "atomics into a [T, H] accumulator) and a finalize kernel rounds it into y")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false",
                     help="skip the CPU oracle leg (used for profiler runs)")
     args = ap.parse_args()

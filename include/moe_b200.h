@@ -20,7 +20,8 @@
  * moe_eplb_plan / moe_eplb_remap / moe_eplb_replicate (replicas of hot
  * experts placed over the logical ranks), and moe_combine_rank_partials /
  * moe_reduce_rank_partials (the masking form: per-rank partial outputs and
- * their rank-ordered sum).
+ * their rank-ordered sum), and moe_ep_* (the exchange of rows between ranks
+ * for expert parallelism over several GPUs).
  *
  * Sources (page title, section):
  *  [EPRT]   "EP: Partition Experts and Route Tokens": "Send tokens to experts
@@ -42,7 +43,9 @@
  *    Slot s = t*k + j is token t's j-th choice.
  *  - All array arguments are DEVICE pointers owned by the caller, row-major,
  *    except where a call says HOST (moe_eplb_plan's arrays, the
- *    phys_to_logical table of moe_eplb_replicate); activation and weight
+ *    phys_to_logical table of moe_eplb_replicate, moe_ep_plan_host's and
+ *    moe_ep_exchange_offsets' arrays, moe_ep_pack's per-destination pointer
+ *    tables); activation and weight
  *    buffers (and the workspace) 16-byte aligned, int32/float32 index and
  *    weight arrays 4-byte aligned.  The library never allocates, frees or
  *    copies to the host, and never synchronises, except moe_get_error.
@@ -165,6 +168,37 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
                         int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * moe_route_count + moe_dispatch_counted -- moe_route and moe_dispatch with
+ * the dispatch's counting moved into the routing kernel.  The router already
+ * holds each token's choices; counting them there (per chunk of slots: the
+ * experts' counts and each slot's stable rank among the chunk's slots of its
+ * expert, into the dispatch workspace) leaves the dispatch kernel only the
+ * scan of the chunk counts, the permutation and the row copy, with no grid
+ * barrier before its copy when the count table is small (chunks x E <= 8192).
+ *
+ * The pair counts in chunks of at most 128 slots (moe_dispatch: 512), so the
+ * routing kernel has a CTA per chunk and a warp per token.
+ *
+ * moe_route_count: exactly moe_route (same ids and weights, bit for bit),
+ * plus that counting into `workspace` (moe_route_count_workspace_bytes(T, k,
+ * E, R) bytes, zero-filled once, as moe_dispatch's).  Ids outside [0, E)
+ * cannot arise from finite logits.
+ * moe_dispatch_counted: moe_dispatch's arguments and results (its workspace
+ * sized by moe_route_count_workspace_bytes), for the topk_ids that
+ * moe_route_count last wrote with this workspace and the same T, k, E, R (it
+ * may be called again on them: the counting is kept).
+ * Counts that do not belong to the ids given never move a row outside its
+ * expert's segment: such slots are dropped and flagged (bit 2).
+ */
+size_t moe_route_count_workspace_bytes(int T, int k, int E, int R);
+moe_status moe_route_count(const float* logits, int T, int E, int k, int R, int32_t* topk_ids, float* topk_w,
+                           void* workspace, size_t workspace_bytes, void* stream);
+moe_status moe_dispatch_counted(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
+                                void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                                int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
+                                int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * moe_dispatch_noalloc -- moe_dispatch for callers that cannot allocate.
  * (The pages have no counterpart: this is a deployment variant of this
  * library's dispatch.)
@@ -256,6 +290,29 @@ moe_status moe_ffn_down(const void* h, int dtype, const void* w_down, const int3
                         int I, int S, void* y_disp, void* stream);
 
 /*
+ * moe_ffn_down_combine + moe_combine_finalize -- moe_ffn_down fused with
+ * moe_combine ([EPRT] "Send tokens ...": results return to their source
+ * tokens; "Return multiple ...": y(t) = sum_j w_j u_j): the down projection's
+ * epilogue multiplies each row's output by its slot's weight and adds it into
+ * a float32 accumulator by token, so y_disp is never written or read.
+ *   row_to_slot [S] int32, topk_w [T, k] float32   from moe_dispatch / moe_route
+ *   y_acc       [T, H] float32: zero on entry to the first call (the finalize
+ *               leaves it zero again); gets  sum_j w[t][j] * (h Wd)[row of t*k+j]
+ * moe_combine_finalize: y[t] = y_acc[t] rounded to bf16, then y_acc = 0.
+ * The additions are float32 atomics (red.global.add.v4.f32): their order,
+ * hence the last bits of y, is not fixed from run to run (moe_combine sums in
+ * j order).  Single-CTA tiles whatever the tiling setting; bf16 only
+ * (MOE_ERR_UNSUPPORTED otherwise).  A row whose slot is outside [0, T*k) is
+ * skipped and flagged (bit 4).  Pays where the accumulator stays in L2 (few
+ * tokens, e.g. decode); elsewhere its T*H*4 bytes of reductions cost more than
+ * the combine they replace.
+ */
+moe_status moe_ffn_down_combine(const void* h, int dtype, const void* w_down, const int32_t* expert_offsets, int E,
+                                int H, int I, int S, const int32_t* row_to_slot, const float* topk_w, int T, int k,
+                                float* y_acc, void* stream);
+moe_status moe_combine_finalize(float* y_acc, int dtype, int T, int H, void* y, void* stream);
+
+/*
  * moe_ffn_gate_up_gather -- moe_ffn_gate_up fused with the row scatter of
  * moe_dispatch ([EPRT] "Send tokens ...": a dispatched row is a copy of its
  * token's row): the A operand of dispatched row r is read straight from x,
@@ -327,6 +384,103 @@ moe_status moe_combine_rank_partials(const void* y_disp, int dtype, const float*
                                     const int32_t* slot_to_row, int T, int k, int H, int E, int R, void* y_part,
                                     void* stream);
 moe_status moe_reduce_rank_partials(const void* y_part, int dtype, int T, int H, int R, void* y, void* stream);
+
+/*
+ * Expert-parallel exchange between ranks -- [EPRT] "Send tokens ...": each
+ * GPU routes its own tokens and sends each token vector to the GPU holding
+ * its selected expert (an exchange by destination with unequal counts);
+ * results return to the source GPU and token, which forms the weighted sum.
+ * "Return multiple ...": input delivery is shared when two selected experts
+ * sit on the same GPU.  [NEURON] "Limitations" 3-4: rank d holds experts
+ * [d*E/R, (d+1)*E/R) (EL = E/R local experts).
+ *
+ * One layer over R ranks (R <= 64), every rank a source and a destination:
+ *   source s:  moe_route; moe_ep_plan; (counts exchange: every rank gets all
+ *              R send_counts vectors); moe_ep_exchange_offsets; moe_ep_pack
+ *              into the destinations' receive buffers (peer memory), or into
+ *              a local buffer for a staged all-to-all;
+ *   (all ranks: barrier, or the all-to-all itself)
+ *   destination d: moe_ep_recv_index over its received rows; the gathering
+ *              gate/up projection (moe_ffn_gate_up_gather with x = received
+ *              rows, row_to_slot from moe_ep_recv_index, k) and moe_ffn_down
+ *              with its EL local experts' weights; moe_combine(y_gemm,
+ *              recv_w, slot_to_row, T_recv, k) gives one partial per received
+ *              row (the weighted sum over the row's local experts); the
+ *              partials of source s (rows [recv_base[s], recv_base[s+1]))
+ *              return to s's return buffer at ret_base[s];
+ *   (barrier)
+ *   source s:  moe_combine(y_ret, ones [T, k], ret_row, T, k) sums each
+ *              token's partials: its output.
+ * The library moves no rows between GPUs by itself except through the peer
+ * pointers given to moe_ep_pack; barriers and the counts exchange belong to
+ * the caller (NCCL, or a host process group).
+ *
+ * moe_ep_plan (device) / moe_ep_plan_host (HOST arrays, no device work): the
+ * send plan of one source rank with T tokens.  One send row per (token t,
+ * destination d holding any of t's experts), ordered by d, then t:
+ *   topk_ids, topk_w [T, k]  from moe_route (global expert ids)
+ *   send_counts  [R]         out: rows for each destination
+ *   send_offsets [R + 1]     out: exclusive prefix sum of send_counts
+ *   slot_send_row [T * k]    out: send row of slot t*k+j's (t, d) pair
+ *   ret_row      [T * k]     out: that row for the first choice of t on each
+ *                            destination, -1 for its other choices there (so
+ *                            a token's partials are each summed once)
+ *   row_token    [T * min(k, R)] out: token of each send row
+ *   row_ids      [T * min(k, R), k] out: the token's local expert ids on the
+ *                            row's destination (id - d*EL), in top-k order,
+ *                            -1 past the last
+ *   row_w        [T * min(k, R), k] float32 out: their weights, 0 past the last
+ *   workspace    moe_ep_plan_workspace_bytes(T, R) bytes (no zeroing needed)
+ * Ids outside [0, E) are dropped (their slots' rows are -1) and flagged
+ * (device: bit 1 of the error word; host: MOE_ERR_DEVICE).  Two kernels.
+ *
+ * moe_ep_exchange_offsets (HOST arrays): from counts [R][R] (row s = source
+ * s's send_counts) for rank `rank`:
+ *   dst_base[d]  = sum_{s < rank} counts[s][d]  (where rank's rows start in
+ *                  d's receive buffer)
+ *   recv_base[s] = sum_{s' < s} counts[s'][rank]  ([R + 1]; recv_base[R]
+ *                  rows are received)
+ *   ret_base[s]  = sum_{d < rank} counts[s][d]  (where rank's partials for
+ *                  source s go in s's return buffer)
+ *
+ * moe_ep_pack: every send row r of destination d goes to
+ *   dst_x[d]   row dst_base[d] + r - send_offsets[d]  (x[row_token[r]])
+ *   dst_ids[d], dst_w[d] at the same row: row_ids[r], row_w[r]
+ * dst_x, dst_ids, dst_w, dst_cap are HOST arrays of R entries (device
+ * pointers, possibly peers' memory; dst_cap[d] rows each); dst_base is a
+ * DEVICE array [R] (moe_ep_exchange_offsets' dst_base, or send_offsets for a
+ * local staging buffer).  A destination row beyond dst_cap[d] is skipped and
+ * flagged (bit 4).  16-byte vector copies, a warp per (row, column slice).
+ *
+ * moe_ep_recv_index: the received rows' counting sort by local expert:
+ *   recv_ids       [T_recv, k]  received row_ids (-1 = padding, never
+ *                               flagged; rows past the received count must
+ *                               be all -1)
+ *   expert_counts  [EL], expert_offsets [EL + 1]  out
+ *   slot_to_row    [T_recv * k] out: GEMM row of (received row q, choice i),
+ *                               -1 for padding
+ *   row_to_slot    [T_recv * k] out: q*k + i of each GEMM row
+ *   workspace      moe_dispatch_workspace_bytes(T_recv, k, EL, 1) bytes,
+ *                  zero-filled once (as moe_dispatch's)
+ * GEMM rows are ordered by (local expert, received row): stable.
+ */
+size_t moe_ep_plan_workspace_bytes(int T, int R);
+moe_status moe_ep_plan(const int32_t* topk_ids, const float* topk_w, int T, int k, int E, int R,
+                       int32_t* send_counts, int32_t* send_offsets, int32_t* slot_send_row, int32_t* ret_row,
+                       int32_t* row_token, int32_t* row_ids, float* row_w, void* workspace, size_t workspace_bytes,
+                       void* stream);
+moe_status moe_ep_plan_host(const int32_t* topk_ids, const float* topk_w, int T, int k, int E, int R,
+                            int32_t* send_counts, int32_t* send_offsets, int32_t* slot_send_row, int32_t* ret_row,
+                            int32_t* row_token, int32_t* row_ids, float* row_w);
+moe_status moe_ep_exchange_offsets(const int32_t* counts, int R, int rank, int32_t* dst_base, int32_t* recv_base,
+                                   int32_t* ret_base);
+moe_status moe_ep_pack(const void* x, int dtype, int T, int H, int k, int R, const int32_t* send_offsets,
+                       const int32_t* dst_base, const int32_t* row_token, const int32_t* row_ids, const float* row_w,
+                       void* const* dst_x, int32_t* const* dst_ids, float* const* dst_w, const int32_t* dst_cap,
+                       void* stream);
+moe_status moe_ep_recv_index(const int32_t* recv_ids, int T_recv, int k, int EL, int32_t* expert_counts,
+                             int32_t* expert_offsets, int32_t* slot_to_row, int32_t* row_to_slot, void* workspace,
+                             size_t workspace_bytes, void* stream);
 
 /*
  * Expert placement with replicas -- an expert-parallel load balancer:

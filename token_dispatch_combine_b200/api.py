@@ -107,13 +107,20 @@ class DispatchOut:
             src_expert_counts=torch.empty((R, E), **i32) if src_counts else None)
 
 
+def moe_route_count_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
+    return int(_native.lib().moe_route_count_workspace_bytes(T, k, E, R))
+
+
 def new_dispatch_workspace(T: int, k: int, E: int, R: int, device) -> torch.Tensor:
-    """Zero-filled workspace of moe_dispatch_workspace_bytes() bytes."""
-    return torch.zeros(moe_dispatch_workspace_bytes(T, k, E, R), dtype=torch.uint8, device=device)
+    """Zero-filled workspace large enough for moe_dispatch and for the counted pair
+    (moe_route_count + moe_dispatch_counted)."""
+    n = max(moe_dispatch_workspace_bytes(T, k, E, R), moe_route_count_workspace_bytes(T, k, E, R))
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def moe_dispatch(x: torch.Tensor | None, topk_ids: torch.Tensor, E: int, R: int, out: DispatchOut,
-                 workspace: torch.Tensor, stream=None, H: int | None = None, dtype=None) -> DispatchOut:
+                 workspace: torch.Tensor, stream=None, H: int | None = None, dtype=None,
+                 _entry: str = "moe_dispatch") -> DispatchOut:
     """Dispatch; with x None and out.x_disp None it is index-only (counts,
     offsets and permutation; no rows move), and H / dtype name the row shape."""
     if x is not None:
@@ -125,15 +132,37 @@ def moe_dispatch(x: torch.Tensor | None, topk_ids: torch.Tensor, E: int, R: int,
             raise ValueError("index-only dispatch needs H and dtype")
     k = topk_ids.shape[1]
     i32 = torch.int32
-    check(_native.lib().moe_dispatch(
+    check(getattr(_native.lib(), _entry)(
         _ptr(x, "x"), _DT[dtype] if dtype in _DT else _dtype(x), T, H, _ptr(topk_ids, "topk_ids", i32), k, E, R,
         _ptr(out.x_disp, "x_disp", dtype),
         _ptr(out.expert_counts, "expert_counts", i32), _ptr(out.expert_offsets, "expert_offsets", i32),
         _ptr(out.rank_counts, "rank_counts", i32), _ptr(out.rank_offsets, "rank_offsets", i32),
         _ptr(out.slot_to_row, "slot_to_row", i32), _ptr(out.row_to_slot, "row_to_slot", i32),
         _ptr(out.src_expert_counts, "src_expert_counts", i32), _ptr(workspace, "workspace", torch.uint8),
-        workspace.numel(), _stream(stream)), "moe_dispatch")
+        workspace.numel(), _stream(stream)), _entry)
     return out
+
+
+def moe_route_count(logits: torch.Tensor, k: int, R: int, workspace: torch.Tensor, topk_ids=None, topk_w=None,
+                    stream=None):
+    """moe_route plus the dispatch's counting into `workspace` (a moe_dispatch workspace for
+    these T, k, E, R): moe_dispatch_counted on the same ids and workspace then skips its counting."""
+    T, E = logits.shape
+    if topk_ids is None:
+        topk_ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    check(_native.lib().moe_route_count(_ptr(logits, "logits", torch.float32), T, E, k, int(R),
+                                        _ptr(topk_ids, "topk_ids", torch.int32), _ptr(topk_w, "topk_w", torch.float32),
+                                        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream)),
+          "moe_route_count")
+    return topk_ids, topk_w
+
+
+def moe_dispatch_counted(x: torch.Tensor | None, topk_ids: torch.Tensor, E: int, R: int, out: DispatchOut,
+                         workspace: torch.Tensor, stream=None, H: int | None = None, dtype=None) -> DispatchOut:
+    """moe_dispatch for the ids moe_route_count last wrote with this workspace (same arguments)."""
+    return moe_dispatch(x, topk_ids, E, R, out, workspace, stream, H, dtype, _entry="moe_dispatch_counted")
 
 
 def moe_ffn_gate_up(x_disp, w_gate, w_up, expert_offsets, h, stream=None):
@@ -153,6 +182,28 @@ def moe_ffn_down(h, w_down, expert_offsets, y_disp, stream=None):
         _ptr(h, "h"), _dtype(h), _ptr(w_down, "w_down", h.dtype), _ptr(expert_offsets, "expert_offsets", torch.int32),
         E, H, I, S, _ptr(y_disp, "y_disp", h.dtype), _stream(stream)), "moe_ffn_down")
     return y_disp
+
+
+def moe_ffn_down_combine(h, w_down, expert_offsets, row_to_slot, topk_w, y_acc, stream=None):
+    """y_acc[t] += sum_j w[t, j] * (h Wd)[row of slot t*k+j]: the down projection with the combine
+    in its epilogue (float32 atomics; y_disp is not formed).  y_acc [T, H] float32, zero on the
+    first call (moe_combine_finalize leaves it zero)."""
+    S, I = h.shape
+    E, _, H = w_down.shape
+    T, k = topk_w.shape
+    check(_native.lib().moe_ffn_down_combine(
+        _ptr(h, "h"), _dtype(h), _ptr(w_down, "w_down", h.dtype), _ptr(expert_offsets, "expert_offsets", torch.int32),
+        E, H, I, S, _ptr(row_to_slot, "row_to_slot", torch.int32), _ptr(topk_w, "topk_w", torch.float32), T, k,
+        _ptr(y_acc, "y_acc", torch.float32), _stream(stream)), "moe_ffn_down_combine")
+    return y_acc
+
+
+def moe_combine_finalize(y_acc, y, stream=None):
+    """y = y_acc rounded to y's dtype (bf16); y_acc zeroed for the next moe_ffn_down_combine."""
+    T, H = y.shape
+    check(_native.lib().moe_combine_finalize(_ptr(y_acc, "y_acc", torch.float32), _dtype(y), T, H, _ptr(y, "y"),
+                                             _stream(stream)), "moe_combine_finalize")
+    return y
 
 
 def moe_ffn_gate_up_gather(x, row_to_slot, k, w_gate, w_up, expert_offsets, h, stream=None):
@@ -198,6 +249,33 @@ def moe_combine(y_disp, topk_w, slot_to_row, y, stream=None):
     check(_native.lib().moe_combine(
         _ptr(y_disp, "y_disp", y.dtype), _dtype(y), _ptr(topk_w, "topk_w", torch.float32),
         _ptr(slot_to_row, "slot_to_row", torch.int32), T, k, H, _ptr(y, "y"), _stream(stream)), "moe_combine")
+    return y
+
+
+def moe_combine_rank_partials(y_disp, topk_w, topk_ids, slot_to_row, E: int, R: int, y_part=None, stream=None):
+    """Masking form of expert parallelism: y_part[r, t] = the w-weighted sum of token t's expert
+    outputs whose expert rank r owns (experts [r*E/R, (r+1)*E/R)), zero where it owns none.
+    Returns y_part [R, T, H] (allocated if not given)."""
+    T, k = topk_w.shape
+    H = y_disp.shape[1]
+    if y_part is None:
+        y_part = torch.empty((R, T, H), dtype=y_disp.dtype, device=y_disp.device)
+    check(_native.lib().moe_combine_rank_partials(
+        _ptr(y_disp, "y_disp"), _dtype(y_disp), _ptr(topk_w, "topk_w", torch.float32),
+        _ptr(topk_ids, "topk_ids", torch.int32), _ptr(slot_to_row, "slot_to_row", torch.int32), T, k, H, int(E),
+        int(R), _ptr(y_part, "y_part", y_disp.dtype), _stream(stream)), "moe_combine_rank_partials")
+    return y_part
+
+
+def moe_reduce_rank_partials(y_part, y=None, stream=None):
+    """y[t] = sum over ranks r (in order) of y_part[r, t]: the reduce-scatter / all-reduce of the
+    masking form, on one GPU."""
+    R, T, H = y_part.shape
+    if y is None:
+        y = torch.empty((T, H), dtype=y_part.dtype, device=y_part.device)
+    check(_native.lib().moe_reduce_rank_partials(_ptr(y_part, "y_part"), _dtype(y_part), T, H, R,
+                                                 _ptr(y, "y", y_part.dtype), _stream(stream)),
+          "moe_reduce_rank_partials")
     return y
 
 
@@ -250,13 +328,17 @@ class MoERoundTrip:
         """gather="auto": bf16 layers with fewer than GATHER_MAX_ROWS_PER_EXPERT rows per expert."""
         return dtype == torch.bfloat16 and T * k < cls.GATHER_MAX_ROWS_PER_EXPERT * E
 
-    def __init__(self, T, H, I, E, k, R, dtype, device="cuda", src_counts=True, gather="auto"):
+    def __init__(self, T, H, I, E, k, R, dtype, device="cuda", src_counts=True, gather="auto", rank_partials=False,
+                 route_counts=True, combine_in_down=False):
         self.T, self.H, self.I, self.E, self.k, self.R = T, H, I, E, k, R
         self.dtype = dtype
         self.device = torch.device(device)
         if gather == "auto":
             gather = self.gathers_by_default(T, k, E, dtype)
         self.gather = bool(gather)
+        # route() also does the dispatch's counting (moe_route_count) and dispatch() reads it
+        # (moe_dispatch_counted); False: moe_route and moe_dispatch
+        self.route_counts = bool(route_counts)
         self._x = None
         S = T * k
         self.topk_ids = torch.empty((T, k), dtype=torch.int32, device=self.device)
@@ -266,16 +348,25 @@ class MoERoundTrip:
         self.h = torch.empty((S, I), dtype=dtype, device=self.device)
         self.y_disp = torch.empty((S, H), dtype=dtype, device=self.device)
         self.y = torch.empty((T, H), dtype=dtype, device=self.device)
+        # the masking form's per-rank partial outputs (combine_masked), [R, T, H]
+        self.y_part = torch.empty((R, T, H), dtype=dtype, device=self.device) if rank_partials else None
+        # combine_in_down: the down projection adds w * output into a float32 [T, H] accumulator
+        # (moe_ffn_down_combine) and a finalize kernel rounds it into y; y_disp is not used (bf16)
+        self.combine_in_down = bool(combine_in_down) and dtype == torch.bfloat16
+        self.y_acc = torch.zeros((T, H), dtype=torch.float32, device=self.device) if self.combine_in_down else None
 
     def route(self, logits, stream=None):
+        if self.route_counts:
+            return moe_route_count(logits, self.k, self.R, self.workspace, self.topk_ids, self.topk_w, stream)
         return moe_route(logits, self.k, self.topk_ids, self.topk_w, stream)
 
     def dispatch(self, x, stream=None):
+        fn = moe_dispatch_counted if self.route_counts else moe_dispatch
         if self.gather:  # the rows stay in x; gate_up reads them there
             self._x = x
-            return moe_dispatch(None, self.topk_ids, self.E, self.R, self.disp, self.workspace, stream,
-                                H=self.H, dtype=self.dtype)
-        return moe_dispatch(x, self.topk_ids, self.E, self.R, self.disp, self.workspace, stream)
+            return fn(None, self.topk_ids, self.E, self.R, self.disp, self.workspace, stream, H=self.H,
+                      dtype=self.dtype)
+        return fn(x, self.topk_ids, self.E, self.R, self.disp, self.workspace, stream)
 
     def gate_up(self, w_gate, w_up, stream=None):
         if self.gather:
@@ -286,10 +377,24 @@ class MoERoundTrip:
         return moe_ffn_gate_up(self.disp.x_disp, w_gate, w_up, self.disp.expert_offsets, self.h, stream)
 
     def down(self, w_down, stream=None):
+        if self.combine_in_down:
+            return moe_ffn_down_combine(self.h, w_down, self.disp.expert_offsets, self.disp.row_to_slot, self.topk_w,
+                                        self.y_acc, stream)
         return moe_ffn_down(self.h, w_down, self.disp.expert_offsets, self.y_disp, stream)
 
     def combine(self, stream=None, y=None):
+        if self.combine_in_down:
+            return moe_combine_finalize(self.y_acc, self.y if y is None else y, stream)
         return moe_combine(self.y_disp, self.topk_w, self.disp.slot_to_row, self.y if y is None else y, stream)
+
+    def combine_masked(self, stream=None, y=None):
+        """The masking form's return path in place of combine: per-rank partial outputs
+        (self.y_part, [R, T, H]) and their rank-ordered sum.  Needs rank_partials=True."""
+        if self.y_part is None:
+            raise RuntimeError("combine_masked needs MoERoundTrip(..., rank_partials=True)")
+        moe_combine_rank_partials(self.y_disp, self.topk_w, self.topk_ids, self.disp.slot_to_row, self.E, self.R,
+                                  self.y_part, stream)
+        return moe_reduce_rank_partials(self.y_part, self.y if y is None else y, stream)
 
     def forward(self, x, logits, w_gate, w_up, w_down, stream=None, y=None):
         self.route(logits, stream)
@@ -297,6 +402,14 @@ class MoERoundTrip:
         self.gate_up(w_gate, w_up, stream)
         self.down(w_down, stream)
         return self.combine(stream, y)
+
+    def forward_masked(self, x, logits, w_gate, w_up, w_down, stream=None, y=None):
+        """forward with the masking form's return path (combine_masked): six kernels."""
+        self.route(logits, stream)
+        self.dispatch(x, stream)
+        self.gate_up(w_gate, w_up, stream)
+        self.down(w_down, stream)
+        return self.combine_masked(stream, y)
 
     KERNELS_PER_FORWARD = 5  # route, dispatch, gate/up, down, combine
 
@@ -393,7 +506,8 @@ class MoEBalancedRoundTrip:
     def __init__(self, T, H, I, E, k, R, slots_per_rank, dtype, device="cuda", gather="auto"):
         self.E, self.k, self.R, self.slots = E, k, R, slots_per_rank
         self.P = R * slots_per_rank
-        self.rt = MoERoundTrip(T, H, I, self.P, k, R, dtype, device=device, gather=gather)
+        # ids are remapped between routing and dispatch: the dispatch counts them itself
+        self.rt = MoERoundTrip(T, H, I, self.P, k, R, dtype, device=device, gather=gather, route_counts=False)
         self.logical_ids = torch.empty((T, k), dtype=torch.int32, device=self.rt.device)
         self.plan = None
         self.w = None

@@ -38,6 +38,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "route.cuh"
 
 namespace moe {
 
@@ -51,9 +52,18 @@ constexpr uint64_t kGridBarrierLimitNs = 1000000000ull;   // 1 s: the limit of e
 // memory, which saves the second grid barrier.
 constexpr size_t kSmallCountTable = 8192;
 
+// Chunk size of the counted pair (moe_route_count / moe_dispatch_counted):
+// small chunks give the routing kernel, a CTA per chunk, a warp per token.
+constexpr int kCountedChunk = 128;
+
+// A small count table is held transposed in shared memory, expert-major with
+// an odd row stride (no bank conflicts on either access pattern).
+__host__ __device__ __forceinline__ int dispatch_table_ld(int nchunks) { return nchunks | 1; }
+
 __host__ __device__ __forceinline__ size_t dispatch_smem_table(int nchunks, int E) {
   const size_t warps = (size_t)kDispatchWarps * E, table = (size_t)nchunks * E;
-  return (table <= kSmallCountTable && table > warps) ? table : warps;
+  const size_t held = (size_t)dispatch_table_ld(nchunks) * E;
+  return (table <= kSmallCountTable && held > warps) ? held : warps;
 }
 
 struct DispatchGeom {
@@ -68,7 +78,8 @@ __host__ __device__ __forceinline__ int src_rank_first_token(int r, int T, int R
   return (int)(((int64_t)r * T + R - 1) / R);
 }
 
-inline DispatchGeom make_dispatch_geom(int T, int k, int E, int R) {
+// max_chunk: kDispatchThreads (moe_dispatch), kCountedChunk (the counted pair).
+inline DispatchGeom make_dispatch_geom(int T, int k, int E, int R, int max_chunk = kDispatchThreads) {
   DispatchGeom g;
   g.T = T;
   g.k = k;
@@ -78,7 +89,7 @@ inline DispatchGeom make_dispatch_geom(int T, int k, int E, int R) {
   const int max_tok = (T + R - 1) / R;  // largest source-rank range
   const int max_slots = max_tok * k;
   int ch = ((max_slots + 31) / 32) * 32;
-  if (ch > kDispatchThreads) ch = kDispatchThreads;
+  if (ch > max_chunk) ch = max_chunk;
   if (ch < 32) ch = 32;
   g.chunk = ch;
   g.cpr = (max_slots + ch - 1) / ch;
@@ -173,6 +184,53 @@ __device__ __forceinline__ bool grid_barrier(const DispatchWs& ws, int* s_ok, ui
   return *s_ok != 0;
 }
 
+// Phase 1 for chunk c: each slot's stable rank among the same-expert slots of
+// the chunk, without atomics (__match_any_sync groups a warp's lanes by
+// expert, popc of the lower peers gives the in-warp rank, a per-expert scan
+// over the CTA's warps adds the earlier warps' counts), into ws.slot_rank; the
+// chunk's per-expert counts into ws.chunk_counts.  id_of(s) is slot s's
+// expert id; ids outside [0, E) are dropped and flagged (a -1 silently when
+// allow_pad).  NW: warps of the block (at least kDispatchWarps, so that
+// every slot of a chunk has a thread); warp_counts: [NW][E] ints of shared
+// memory.
+template <int NW, typename IdOf>
+__device__ __forceinline__ void count_chunk(const DispatchGeom& g, int c, const DispatchWs& ws, int32_t* warp_counts,
+                                            int allow_pad, IdOf id_of) {
+  static_assert(NW >= kDispatchWarps, "a thread per slot of a chunk");
+  constexpr int NT = NW * 32;
+  const int warp = threadIdx.x >> 5, lane = (int)lane_id();
+  int s0, s1;
+  chunk_slot_range(g, c, s0, s1);
+  for (int i = threadIdx.x; i < NW * g.E; i += NT) warp_counts[i] = 0;
+  __syncthreads();
+  const int s = s0 + (int)threadIdx.x;
+  int e = -2;  // -2: no slot; -1: bad id
+  if (s < s1) {
+    e = id_of(s);
+    if (e < 0 || e >= g.E) {
+      if (!(allow_pad && e == -1)) flag_error(kErrBadId);  // -1 is padding where allowed
+      e = -1;
+    }
+  }
+  const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+  const int rank_in_warp = __popc(peers & ((1u << lane) - 1u));
+  if (e >= 0 && lane == __ffs(peers) - 1) warp_counts[warp * g.E + e] = __popc(peers);
+  __syncthreads();
+  for (int xx = threadIdx.x; xx < g.E; xx += NT) {  // exclusive scan over warps, per expert
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const int v = warp_counts[w * g.E + xx];
+      warp_counts[w * g.E + xx] = run;
+      run += v;
+    }
+    ws.chunk_counts[(size_t)c * g.E + xx] = run;
+  }
+  __syncthreads();
+  if (s < s1) ws.slot_rank[s] = (e >= 0) ? warp_counts[warp * g.E + e] + rank_in_warp : -1;
+  __syncthreads();  // warp_counts is reused by the next chunk
+}
+
 // Last step of every CTA on every path (thread 0 only, after its last barrier
 // operation): arrive on the exit counter; the last CTA out zeroes the arrival
 // and exit counters.  A barrier that timed out leaves a partial arrival count
@@ -193,7 +251,8 @@ __device__ __forceinline__ void dispatch_exit(const DispatchWs& ws) {
 template <typename T>
 __device__ __forceinline__ void dispatch_phases(
     const DispatchGeom& g, int H, int nslices, int tpc, const T* __restrict__ x, const int32_t* __restrict__ ids,
-    const DispatchWs& ws, uint64_t limit_ns, T* __restrict__ x_disp, int32_t* __restrict__ expert_counts,
+    const DispatchWs& ws, uint64_t limit_ns, int allow_pad, int counted, T* __restrict__ x_disp,
+    int32_t* __restrict__ expert_counts,
     int32_t* __restrict__ expert_offsets, int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets,
     int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
   extern __shared__ int32_t smem_i32[];
@@ -201,7 +260,8 @@ __device__ __forceinline__ void dispatch_phases(
   int32_t* offs = smem_i32 + dispatch_smem_table(g.nchunks, g.E);     // [E + 1]
   int32_t* s_rows = offs + g.E + 1;                                    // [kDispatchThreads]
   const bool small_table = (size_t)g.nchunks * g.E <= kSmallCountTable;
-  int32_t* cbase = smem_i32;  // small_table: [nchunks][E] chunk bases (reuses warp_counts)
+  const int ld = dispatch_table_ld(g.nchunks);
+  int32_t* cbase = smem_i32;  // small_table: [E][ld] chunk bases, expert-major (reuses warp_counts)
   __shared__ int s_ok;
   // ---- this CTA's tokens [tb, te): ask L2 for their rows of x.  A prefetch
   // changes no data, so it may run before the previous kernel has finished.
@@ -238,54 +298,39 @@ __device__ __forceinline__ void dispatch_phases(
     }
   }
 
-  // ---- phase 1: per-chunk stable ranks and counts
-  for (int c = blockIdx.x; c < g.nchunks; c += gridDim.x) {
-    int s0, s1;
-    chunk_slot_range(g, c, s0, s1);
-    for (int i = threadIdx.x; i < kDispatchWarps * g.E; i += kDispatchThreads) warp_counts[i] = 0;
-    __syncthreads();
-    const int s = s0 + (int)threadIdx.x;
-    int e = -2;  // -2: no slot; -1: bad id
-    if (s < s1) {
-      e = __ldg(ids + s);
-      if (e < 0 || e >= g.E) {
-        flag_error(kErrBadId);
-        e = -1;
-      }
-    }
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
-    const int rank_in_warp = __popc(peers & ((1u << lane) - 1u));
-    if (e >= 0 && lane == __ffs(peers) - 1) warp_counts[warp * g.E + e] = __popc(peers);
-    __syncthreads();
-    for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) {  // exclusive scan over warps, per expert
-      int run = 0;
-#pragma unroll
-      for (int w = 0; w < kDispatchWarps; ++w) {
-        const int v = warp_counts[w * g.E + xx];
-        warp_counts[w * g.E + xx] = run;
-        run += v;
-      }
-      ws.chunk_counts[(size_t)c * g.E + xx] = run;
-    }
-    __syncthreads();
-    if (s < s1) ws.slot_rank[s] = (e >= 0) ? warp_counts[warp * g.E + e] + rank_in_warp : -1;
-    __syncthreads();  // warp_counts is reused by the next chunk
+  // ---- phase 1: per-chunk stable ranks and counts (already in the workspace when `counted`:
+  // the routing kernel did them, route_count_kernel)
+  if (!counted) {
+    for (int c = blockIdx.x; c < g.nchunks; c += gridDim.x)
+      count_chunk<kDispatchWarps>(g, c, ws, warp_counts, allow_pad, [&](int s) { return __ldg(ids + s); });
+    if (!grid_barrier(ws, &s_ok, limit_ns)) return;
   }
-  if (!grid_barrier(ws, &s_ok, limit_ns)) return;
 
   if (small_table) {
     // ---- phase 2 (small count table): every CTA scans the whole table itself
-    for (int i = threadIdx.x; i < g.nchunks * g.E; i += kDispatchThreads) cbase[i] = __ldcg(ws.chunk_counts + i);
+    for (int i = threadIdx.x; i < g.nchunks * g.E; i += kDispatchThreads) {  // transposed into shared memory
+      const int c = i / g.E, xx = i - c * g.E;
+      cbase[xx * ld + c] = __ldcg(ws.chunk_counts + i);
+    }
     __syncthreads();
-    for (int xx = threadIdx.x; xx < g.E; xx += kDispatchThreads) {  // thread per expert, prefix over chunks
-      int run = 0;
-      for (int c = 0; c < g.nchunks; ++c) {
-        const int v = cbase[c * g.E + xx];
-        cbase[c * g.E + xx] = run;
-        run += v;
+    for (int xx = warp; xx < g.E; xx += kDispatchWarps) {  // warp per expert, prefix over chunks
+      int carry = 0;
+      for (int base = 0; base < g.nchunks; base += 32) {
+        const int c = base + lane;
+        const int v = (c < g.nchunks) ? cbase[xx * ld + c] : 0;
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+          if (lane >= d) incl += y;
+        }
+        if (c < g.nchunks) cbase[xx * ld + c] = carry + incl - v;
+        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
       }
-      offs[xx] = run;
-      if (blockIdx.x == 0) expert_counts[xx] = run;
+      if (lane == 0) {
+        offs[xx] = carry;
+        if (blockIdx.x == 0) expert_counts[xx] = carry;
+      }
     }
   } else {
   // ---- phase 2a: one warp per expert, prefix over chunks
@@ -334,19 +379,21 @@ __device__ __forceinline__ void dispatch_phases(
   if (blockIdx.x == 0) {
     for (int xx = threadIdx.x; xx <= g.E; xx += kDispatchThreads) expert_offsets[xx] = offs[xx];
     const int EL = g.E / g.R;
-    for (int r = threadIdx.x; r < g.R; r += kDispatchThreads) {
-      rank_counts[r] = offs[(r + 1) * EL] - offs[r * EL];
-      rank_offsets[r] = offs[r * EL];
+    if (rank_counts != nullptr) {  // (NULL only from internal one-rank calls)
+      for (int r = threadIdx.x; r < g.R; r += kDispatchThreads) {
+        rank_counts[r] = offs[(r + 1) * EL] - offs[r * EL];
+        rank_offsets[r] = offs[r * EL];
+      }
+      if (threadIdx.x == 0) rank_offsets[g.R] = placed;
     }
-    if (threadIdx.x == 0) rank_offsets[g.R] = placed;
   }
   if (src_expert_counts) {  // a source rank's chunks are contiguous: differences of the chunk bases
     if (small_table) {
       if (blockIdx.x == 0) {
         for (int i = threadIdx.x; i < g.R * g.E; i += kDispatchThreads) {
           const int r = i / g.E, xx = i - r * g.E;
-          const int lo = cbase[(r * g.cpr) * g.E + xx];
-          const int hi = (r + 1 < g.R) ? cbase[((r + 1) * g.cpr) * g.E + xx] : offs[xx + 1] - offs[xx];
+          const int lo = cbase[xx * ld + r * g.cpr];
+          const int hi = (r + 1 < g.R) ? cbase[xx * ld + (r + 1) * g.cpr] : offs[xx + 1] - offs[xx];
           src_expert_counts[i] = hi - lo;
         }
       }
@@ -374,8 +421,11 @@ __device__ __forceinline__ void dispatch_phases(
       int row = -1;
       if (e >= 0 && e < g.E && rk >= 0) {
         const int c = chunk_of_slot(g, s);
-        const size_t cb = (size_t)c * g.E + e;
-        row = offs[e] + (small_table ? cbase[cb] : __ldcg(ws.chunk_base + cb)) + rk;
+        row = offs[e] + (small_table ? cbase[e * ld + c] : __ldcg(ws.chunk_base + (size_t)c * g.E + e)) + rk;
+        if (row >= offs[e + 1]) {  // counts that do not belong to these ids: never leave the segment
+          flag_error(kErrBadOffsets);
+          row = -1;
+        }
       }
       s_rows[threadIdx.x] = row;
       slot_to_row[s] = row;
@@ -415,20 +465,123 @@ __device__ __forceinline__ void dispatch_phases(
 template <typename T>
 __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
     DispatchGeom g, int H, int nslices, int tpc, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
-    uint64_t limit_ns, T* __restrict__ x_disp, int32_t* __restrict__ expert_counts, int32_t* __restrict__ expert_offsets,
-    int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets, int32_t* __restrict__ slot_to_row,
-    int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
-  dispatch_phases<T>(g, H, nslices, tpc, x, ids, ws, limit_ns, x_disp, expert_counts, expert_offsets, rank_counts,
-                     rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
+    uint64_t limit_ns, int allow_pad, int counted, T* __restrict__ x_disp, int32_t* __restrict__ expert_counts,
+    int32_t* __restrict__ expert_offsets, int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets,
+    int32_t* __restrict__ slot_to_row, int32_t* __restrict__ row_to_slot, int32_t* __restrict__ src_expert_counts) {
+  dispatch_phases<T>(g, H, nslices, tpc, x, ids, ws, limit_ns, allow_pad, counted, x_disp, expert_counts,
+                     expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
   dispatch_exit(ws);
 }
 
-// limit_ns bounds each grid-barrier wait (kGridBarrierLimitNs for moe_dispatch).
+// moe_route_count: the routing of moe_route fused with phase 1 of the
+// dispatch.  One CTA per dispatch chunk (the same geometry, so the counts
+// land where a counted dispatch reads them): its warps route the tokens that
+// have slots in the chunk (a warp per token, warp_topk_softmax; a token whose
+// slots straddle two chunks is routed by both, identically), write the
+// chunk's slots of topk_ids / topk_w and keep their ids in shared memory;
+// then count_chunk ranks and counts the chunk.  Each warp loads the logits of
+// its next token before routing the current one (E <= 256).
+// 1024 threads (512 above 256 experts, whose logits take twice the
+// registers): that many routing warps, then the counting with a thread per
+// slot.  Dynamic shared memory: warp_counts[warps][E], then ids[chunk].
+template <int VPL>
+struct RouteCountCfg {
+  static constexpr int kThreads = VPL >= 16 ? 512 : 1024;
+  static constexpr int kWarps = kThreads / 32;
+};
+template <int VPL>
+__global__ void __launch_bounds__(RouteCountCfg<VPL>::kThreads) route_count_kernel(DispatchGeom g,
+                                                                                  const float* __restrict__ logits,
+                                                                                  int32_t* __restrict__ topk_ids,
+                                                                                  float* __restrict__ topk_w,
+                                                                                  DispatchWs ws) {
+  constexpr int kRouteCountWarps = RouteCountCfg<VPL>::kWarps;
+  extern __shared__ int32_t smem_i32[];
+  int32_t* warp_counts = smem_i32;
+  int32_t* s_ids = smem_i32 + kRouteCountWarps * g.E;
+  pdl_wait();
+  pdl_trigger();
+  const int c = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = (int)lane_id();
+  int s0, s1;
+  chunk_slot_range(g, c, s0, s1);
+  const int t0 = s0 / g.k, t1 = s1 > s0 ? (s1 + g.k - 1) / g.k : t0;
+  float val[VPL], nval[VPL];
+  auto load = [&](int t, float (&v)[VPL]) {
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) {
+      const int e = lane + 32 * q;
+      v[q] = (t < t1 && e < g.E) ? __ldg(logits + (size_t)t * g.E + e) : 0.0f;
+    }
+  };
+  constexpr bool kPrefetch = VPL <= 8;  // (more experts: the second register set would spill)
+  if (kPrefetch) load(t0 + warp, val);
+  for (int t = t0 + warp; t < t1; t += kRouteCountWarps) {
+    if (kPrefetch) load(t + kRouteCountWarps, nval);  // the next token's logits in flight while this one is routed
+    else load(t, val);
+    uint32_t key[VPL];
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) key[q] = (lane + 32 * q < g.E) ? logit_order_key(val[q]) : 0u;
+    int my_id;
+    float my_w;
+    warp_topk_softmax<VPL>(key, val, g.k, lane, my_id, my_w);
+    const int s = t * g.k + lane;
+    if (lane < g.k && s >= s0 && s < s1) {
+      topk_ids[s] = my_id;
+      topk_w[s] = my_w;
+      s_ids[s - s0] = my_id;
+    }
+    if (kPrefetch) {
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) val[q] = nval[q];
+    }
+  }
+  __syncthreads();
+  count_chunk<kRouteCountWarps>(g, c, ws, warp_counts, 0, [&](int s) { return s_ids[s - s0]; });
+}
+
+inline cudaError_t launch_route_count(const DispatchGeom& g, const float* logits, int32_t* ids, float* w,
+                                      void* workspace, cudaStream_t stream) {
+  if (g.T == 0) return cudaSuccess;
+  const DispatchWs ws = dispatch_ws_carve(workspace, g);
+  const int vpl = (g.E + 31) / 32;
+  const int dev = current_device();
+  cudaError_t err = cudaSuccess;
+#define MOE_ROUTE_COUNT_CASE(V)                                                                              \
+  case V: {                                                                                                  \
+    constexpr int NW = RouteCountCfg<V>::kWarps;                                                             \
+    const size_t smem = sizeof(int32_t) * ((size_t)NW * g.E + kDispatchThreads);                            \
+    static PerDeviceOnce attr_once; /* shared memory for the largest E of this case */                      \
+    err = attr_once.run(dev, [&] {                                                                           \
+      return cudaFuncSetAttribute(route_count_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
+                                  (int)(sizeof(int32_t) * ((size_t)NW * 32 * V + kDispatchThreads)));        \
+    });                                                                                                      \
+    if (err == cudaSuccess)                                                                                  \
+      err = launch_pdl(route_count_kernel<V>, dim3(g.nchunks), dim3(NW * 32), smem, stream, g, logits, ids, w, ws); \
+    break;                                                                                                   \
+  }
+  switch (vpl <= 1 ? 1 : vpl <= 2 ? 2 : vpl <= 4 ? 4 : vpl <= 8 ? 8 : vpl <= 16 ? 16 : 32) {
+    MOE_ROUTE_COUNT_CASE(1)
+    MOE_ROUTE_COUNT_CASE(2)
+    MOE_ROUTE_COUNT_CASE(4)
+    MOE_ROUTE_COUNT_CASE(8)
+    MOE_ROUTE_COUNT_CASE(16)
+    MOE_ROUTE_COUNT_CASE(32)
+  }
+#undef MOE_ROUTE_COUNT_CASE
+  return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+// limit_ns bounds each grid-barrier wait (kGridBarrierLimitNs for moe_dispatch).  allow_pad:
+// an id of -1 is padding (dropped like a bad id, but not flagged).  counted: phase 1's counts
+// and ranks are already in the workspace (route_count_kernel), so phase 1 and its barrier
+// are skipped.
 template <typename T>
 cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int32_t* ids, void* workspace,
                             T* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
                             int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
-                            int32_t* src_expert_counts, cudaStream_t stream, uint64_t limit_ns = kGridBarrierLimitNs) {
+                            int32_t* src_expert_counts, cudaStream_t stream, uint64_t limit_ns = kGridBarrierLimitNs,
+                            bool allow_pad = false, bool counted = false) {
   DispatchWs ws = dispatch_ws_carve(workspace, g);
   auto kern = dispatch_kernel<T>;
   const size_t smem = sizeof(int32_t) * (dispatch_smem_table(g.nchunks, g.E) + g.E + 1 + kDispatchThreads);
@@ -437,6 +590,7 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   cudaError_t err = attr_once.run(dev, [&] {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)(sizeof(int32_t) * (dispatch_smem_table(1, 1024) + 1025 + kDispatchThreads)));
+    // (the largest need: the [16][1024] warp counts; a small table is at most 8192 + E entries)
   });
   if (err != cudaSuccess) return err;
   // Co-residency bound of the cooperative grid for this shared-memory size.
@@ -472,8 +626,9 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = MOE_PDL ? 2 : 1;
-  err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, tpc, x, ids, ws, limit_ns, x_disp, expert_counts, expert_offsets,
-                           rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts);
+  err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, tpc, x, ids, ws, limit_ns, (int)allow_pad, (int)counted, x_disp,
+                           expert_counts, expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
+                           src_expert_counts);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

@@ -276,6 +276,13 @@ struct Params {
   const int32_t* gather_rows;  // [S] row_to_slot
   int gather_k, gather_T;
   const void* gather_x;        // [gather_T, K] bf16
+  // Down projection with the combine in its epilogue (single-CTA tiles only):
+  // row r's output, times comb_w[s], is added (float32 atomics) into
+  // comb_acc[s / comb_k] for its slot s = comb_rows[r]; `out` is not written.
+  const int32_t* comb_rows;  // [S] row_to_slot
+  const float* comb_w;       // [comb_T * comb_k] topk_w
+  float* comb_acc;           // [comb_T, N] float32
+  int comb_k, comb_T;
 };
 
 // ---- A-row gather (dispatch fused into the gate/up projection)
@@ -678,6 +685,18 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
       const uint32_t t_base = tmem_base + (uint32_t)acc * kAccStride + ((uint32_t)(q * 32) << 16);
       __nv_bfloat16* out_row = p.out + (size_t)row * p.N;
       constexpr int NCHUNK = (BN + 31) / 32;
+      // combine in the epilogue: this row's slot, weight and token row of the accumulator
+      float comb_wt = 0.0f;
+      float* comb_row = nullptr;
+      if (!GATEUP && p.comb_acc != nullptr && row_ok) {
+        const int s = __ldg(p.comb_rows + row);
+        if (s >= 0 && s < p.comb_T * p.comb_k) {
+          comb_wt = __ldg(p.comb_w + s);
+          comb_row = p.comb_acc + (size_t)(s / p.comb_k) * p.N;
+        } else {
+          flag_error(kErrBadRow);
+        }
+      }
 #pragma unroll 1
       for (int c = 0; c < NCHUNK; ++c) {
         uint32_t r0[32];
@@ -698,7 +717,18 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r0[i]);
         }
-        if (row_ok) {
+        if (!GATEUP && p.comb_acc != nullptr) {
+          if (comb_row != nullptr) {
+#pragma unroll
+            for (int g4 = 0; g4 < 8; ++g4) {
+              const int col = n0 + c * 32 + g4 * 4;
+              if (c * 32 + g4 * 4 < BN && col < p.N)
+                atomicAdd(reinterpret_cast<float4*>(comb_row + col),
+                          make_float4(comb_wt * v[g4 * 4 + 0], comb_wt * v[g4 * 4 + 1], comb_wt * v[g4 * 4 + 2],
+                                      comb_wt * v[g4 * 4 + 3]));
+            }
+          }
+        } else if (row_ok) {
 #pragma unroll
           for (int g8 = 0; g8 < 4; ++g8) {
             const int col = n0 + c * 32 + g8 * 8;
@@ -723,6 +753,25 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Second half of the combine done in the down projection's epilogue: y = the
+// accumulator rounded to bf16, and the accumulator zeroed for the next call.
+// A thread per 8 columns.
+__global__ void __launch_bounds__(256) combine_finalize_kernel(float* __restrict__ acc, size_t n8,
+                                                               __nv_bfloat16* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+    float4* a = reinterpret_cast<float4*>(acc) + 2 * i;
+    const float4 lo = __ldcg(a), hi = __ldcg(a + 1);
+    const uint4 w = make_uint4(pack_bf16x2(lo.x, lo.y), pack_bf16x2(lo.z, lo.w), pack_bf16x2(hi.x, hi.y),
+                               pack_bf16x2(hi.z, hi.w));
+    st_v4(y + 8 * i, w);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    a[0] = z;
+    a[1] = z;
   }
 }
 
@@ -836,9 +885,11 @@ inline cudaError_t launch_gate_up_gather(const void* x, int T, const int32_t* ro
   return launch_tc<true, 128, 4, true>(tg, tg, tu, p, stream);
 }
 
-// y_disp = h Wd; n-tile width chosen to cover H with the least padding
+// y_disp = h Wd; n-tile width chosen to cover H with the least padding.
+// With `comb` (comb_rows, comb_w, comb_acc, comb_k, comb_T set) the epilogue
+// adds w * (h Wd) into comb_acc by token instead of writing y.
 inline cudaError_t launch_down(const void* h, const void* wd, const int32_t* off, int E, int H, int I, int S,
-                               void* y, cudaStream_t stream) {
+                               void* y, cudaStream_t stream, const Params* comb = nullptr) {
   if (S == 0) return cudaSuccess;
   CUtensorMap ta, tb;
   if (!make_tmap_act(&ta, h, S, I) || !make_tmap_weight(&tb, wd, E, I, H)) return cudaErrorInvalidValue;
@@ -858,6 +909,13 @@ inline cudaError_t launch_down(const void* h, const void* wd, const int32_t* off
   }
   if (MOE_TC_DOWN_BN > 0) best = MOE_TC_DOWN_BN;
   Params p{off, E, S, I, H, (H + best - 1) / best, reinterpret_cast<__nv_bfloat16*>(y), nullptr, 1, 0, nullptr};
+  if (comb != nullptr) {
+    p.comb_rows = comb->comb_rows;
+    p.comb_w = comb->comb_w;
+    p.comb_acc = comb->comb_acc;
+    p.comb_k = comb->comb_k;
+    p.comb_T = comb->comb_T;
+  }
   switch (best) {
     case 256:
       return launch_tc<false, 256, 4>(ta, tb, tb, p, stream);
@@ -866,6 +924,19 @@ inline cudaError_t launch_down(const void* h, const void* wd, const int32_t* off
     default:
       return launch_tc<false, 128, 6>(ta, tb, tb, p, stream);
   }
+}
+
+inline cudaError_t launch_combine_finalize(float* acc, int T, int H, void* y, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const size_t n8 = (size_t)T * H / 8;
+  int sms = 0;
+  cudaError_t err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, current_device());
+  if (err != cudaSuccess) return err;
+  size_t blocks = (n8 + 255) / 256;
+  if (blocks > (size_t)sms * 8) blocks = (size_t)sms * 8;
+  err = launch_pdl(combine_finalize_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, acc, n8,
+                   reinterpret_cast<__nv_bfloat16*>(y));
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace tc

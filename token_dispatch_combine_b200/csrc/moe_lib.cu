@@ -17,6 +17,7 @@
 #include "ffn_tc.cuh"
 #include "ffn_tc2.cuh"
 #include "route.cuh"
+#include "ep.cuh"
 #include "eplb.cuh"
 #include "masked.cuh"
 #include "router.cuh"
@@ -162,7 +163,7 @@ moe_status check_dispatch(const void* x, int dtype, int T, int H, const int32_t*
                           const void* x_disp, const int32_t* expert_counts, const int32_t* expert_offsets,
                           const int32_t* rank_counts, const int32_t* rank_offsets, const int32_t* slot_to_row,
                           const int32_t* row_to_slot, const int32_t* src_expert_counts, bool check_workspace,
-                          const void* workspace, size_t workspace_bytes) {
+                          const void* workspace, size_t workspace_bytes, int max_chunk = moe::kDispatchThreads) {
   const size_t es = dtype_size(dtype);
   MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
   MOE_REQUIRE(T >= 0, "T must be >= 0");
@@ -178,8 +179,9 @@ moe_status check_dispatch(const void* x, int dtype, int T, int H, const int32_t*
   MOE_REQUIRE(src_expert_counts == nullptr || aligned(src_expert_counts, 4), "src_expert_counts misaligned");
   if (check_workspace) {
     MOE_REQUIRE_PTR(workspace, 16, "workspace");
-    MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(moe::make_dispatch_geom(T, k, E, R)),
-                "workspace_bytes smaller than moe_dispatch_workspace_bytes()");
+    MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(moe::make_dispatch_geom(T, k, E, R, max_chunk)),
+                max_chunk == moe::kDispatchThreads ? "workspace_bytes smaller than moe_dispatch_workspace_bytes()"
+                                                   : "workspace_bytes smaller than moe_route_count_workspace_bytes()");
   }
   MOE_REQUIRE((x == nullptr) == (x_disp == nullptr),
               "x and x_disp must both be given, or both be NULL (index-only dispatch)");
@@ -200,15 +202,16 @@ cudaError_t enqueue_dispatch(const void* x, int dtype, int T, int H, const int32
                              void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
                              int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
                              int32_t* src_expert_counts, void* workspace, cudaStream_t s,
-                             uint64_t limit_ns = moe::kGridBarrierLimitNs) {
-  const moe::DispatchGeom g = moe::make_dispatch_geom(T, k, E, R);
+                             uint64_t limit_ns = moe::kGridBarrierLimitNs, bool counted = false) {
+  const moe::DispatchGeom g =
+      moe::make_dispatch_geom(T, k, E, R, counted ? moe::kCountedChunk : moe::kDispatchThreads);
   if (dtype == MOE_BF16)
     return moe::launch_dispatch(g, H, (const __nv_bfloat16*)x, topk_ids, workspace, (__nv_bfloat16*)x_disp,
                                 expert_counts, expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
-                                src_expert_counts, s, limit_ns);
+                                src_expert_counts, s, limit_ns, false, counted);
   return moe::launch_dispatch(g, H, (const float*)x, topk_ids, workspace, (float*)x_disp, expert_counts,
                               expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts,
-                              s, limit_ns);
+                              s, limit_ns, false, counted);
 }
 
 }  // namespace
@@ -227,6 +230,45 @@ moe_status moe_dispatch(const void* x, int dtype, int T, int H, const int32_t* t
                                       rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts,
                                       workspace, (cudaStream_t)stream),
                      "moe_dispatch");
+}
+
+size_t moe_route_count_workspace_bytes(int T, int k, int E, int R) {
+  if (T < 0 || k < 1 || E < 1 || R < 1) return 0;
+  return moe::dispatch_ws_bytes(moe::make_dispatch_geom(T, k, E, R, moe::kCountedChunk));
+}
+
+moe_status moe_route_count(const float* logits, int T, int E, int k, int R, int32_t* topk_ids, float* topk_w,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  moe_status st = check_k_e(k, E);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(R >= 1 && E % R == 0, "R must be >= 1 and divide E");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  MOE_REQUIRE_PTR(workspace, 16, "workspace");
+  const moe::DispatchGeom g = moe::make_dispatch_geom(T, k, E, R, moe::kCountedChunk);
+  MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(g),
+              "workspace_bytes smaller than moe_route_count_workspace_bytes()");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(logits, 4, "logits");
+  MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
+  MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
+  return cuda_status(moe::launch_route_count(g, logits, topk_ids, topk_w, workspace, (cudaStream_t)stream),
+                     "moe_route_count");
+}
+
+moe_status moe_dispatch_counted(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k, int E, int R,
+                                void* x_disp, int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                                int32_t* rank_offsets, int32_t* slot_to_row, int32_t* row_to_slot,
+                                int32_t* src_expert_counts, void* workspace, size_t workspace_bytes, void* stream) {
+  moe_status st = check_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                 rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts, true,
+                                 workspace, workspace_bytes, moe::kCountedChunk);
+  if (st != MOE_OK) return st;
+  return cuda_status(enqueue_dispatch(x, dtype, T, H, topk_ids, k, E, R, x_disp, expert_counts, expert_offsets,
+                                      rank_counts, rank_offsets, slot_to_row, row_to_slot, src_expert_counts,
+                                      workspace, (cudaStream_t)stream, moe::kGridBarrierLimitNs,
+                                      /*counted=*/T > 0),  // no tokens: nothing was counted, count the empty chunks
+                     "moe_dispatch_counted");
 }
 
 moe_status moe_selftest_dispatch_timeout(const void* x, int dtype, int T, int H, const int32_t* topk_ids, int k,
@@ -422,6 +464,39 @@ moe_status moe_ffn_down(const void* h, int dtype, const void* w_down, const int3
   return cuda_status(err, "moe_ffn_down");
 }
 
+moe_status moe_ffn_down_combine(const void* h, int dtype, const void* w_down, const int32_t* expert_offsets, int E,
+                                int H, int I, int S, const int32_t* row_to_slot, const float* topk_w, int T, int k,
+                                float* y_acc, void* stream) {
+  moe_status st = check_ffn(dtype, E, H, I, S, h, "h", expert_offsets);
+  if (st != MOE_OK) return st;
+  if (dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "moe_ffn_down_combine: bf16 only");
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= 8, "T >= 0 and k in [1, 8] are required");
+  MOE_REQUIRE((long long)T * k < (1LL << 31) && S <= T * k, "S must be <= T * k < 2^31");
+  if (S == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(w_down, 16, "w_down");
+  MOE_REQUIRE_PTR(row_to_slot, 4, "row_to_slot");
+  MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
+  MOE_REQUIRE_PTR(y_acc, 16, "y_acc");
+  moe::tc::Params comb = {};
+  comb.comb_rows = row_to_slot;
+  comb.comb_w = topk_w;
+  comb.comb_acc = y_acc;
+  comb.comb_k = k;
+  comb.comb_T = T;
+  return cuda_status(moe::tc::launch_down(h, w_down, expert_offsets, E, H, I, S, nullptr, (cudaStream_t)stream, &comb),
+                     "moe_ffn_down_combine");
+}
+
+moe_status moe_combine_finalize(float* y_acc, int dtype, int T, int H, void* y, void* stream) {
+  MOE_REQUIRE(dtype == MOE_BF16 || dtype == MOE_F32, "dtype must be MOE_F32 or MOE_BF16");
+  if (dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "moe_combine_finalize: bf16 only");
+  MOE_REQUIRE(T >= 0 && H >= 8 && H % 8 == 0, "T >= 0 and H a positive multiple of 8 are required");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(y_acc, 16, "y_acc");
+  MOE_REQUIRE_PTR(y, 16, "y");
+  return cuda_status(moe::tc::launch_combine_finalize(y_acc, T, H, y, (cudaStream_t)stream), "moe_combine_finalize");
+}
+
 moe_status moe_expert_ffn(const void* x_disp, int dtype, const void* w_gate, const void* w_up,
                           const void* w_down, const int32_t* expert_offsets, int E, int H, int I, int S, void* h,
                           void* y_disp, void* stream) {
@@ -533,6 +608,146 @@ moe_status moe_reduce_rank_partials(const void* y_part, int dtype, int T, int H,
   else
     err = moe::launch_reduce_ranks((const float*)y_part, T, H, R, (float*)y, s);
   return cuda_status(err, "moe_reduce_rank_partials");
+}
+
+static moe_status check_ep_plan(const int32_t* topk_ids, const float* topk_w, int T, int k, int E, int R,
+                                const int32_t* send_counts, const int32_t* send_offsets, const int32_t* slot_send_row,
+                                const int32_t* ret_row, const int32_t* row_token, const int32_t* row_ids,
+                                const float* row_w) {
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  moe_status st = check_k_e(k, E);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(R >= 1 && R <= moe::kEpMaxRanks && E % R == 0, "R must be in [1, 64] and divide E");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  MOE_REQUIRE_PTR(send_counts, 4, "send_counts");
+  MOE_REQUIRE_PTR(send_offsets, 4, "send_offsets");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(topk_ids, 4, "topk_ids");
+  MOE_REQUIRE_PTR(topk_w, 4, "topk_w");
+  MOE_REQUIRE_PTR(slot_send_row, 4, "slot_send_row");
+  MOE_REQUIRE_PTR(ret_row, 4, "ret_row");
+  MOE_REQUIRE_PTR(row_token, 4, "row_token");
+  MOE_REQUIRE_PTR(row_ids, 4, "row_ids");
+  MOE_REQUIRE_PTR(row_w, 4, "row_w");
+  return MOE_OK;
+}
+
+size_t moe_ep_plan_workspace_bytes(int T, int R) {
+  if (T < 0 || R < 1) return 0;
+  return moe::ep_plan_ws_bytes(T, R);
+}
+
+moe_status moe_ep_plan(const int32_t* topk_ids, const float* topk_w, int T, int k, int E, int R,
+                       int32_t* send_counts, int32_t* send_offsets, int32_t* slot_send_row, int32_t* ret_row,
+                       int32_t* row_token, int32_t* row_ids, float* row_w, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  moe_status st = check_ep_plan(topk_ids, topk_w, T, k, E, R, send_counts, send_offsets, slot_send_row, ret_row,
+                                row_token, row_ids, row_w);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (T == 0) {  // nothing to send: zero counts and offsets
+    cudaError_t err = cudaMemsetAsync(send_counts, 0, sizeof(int32_t) * R, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(send_offsets, 0, sizeof(int32_t) * (R + 1), s);
+    return cuda_status(err, "moe_ep_plan");
+  }
+  MOE_REQUIRE_PTR(workspace, 16, "workspace");
+  MOE_REQUIRE(workspace_bytes >= moe::ep_plan_ws_bytes(T, R), "workspace_bytes smaller than moe_ep_plan_workspace_bytes()");
+  const moe::EpPlanArgs a = moe::ep_plan_args(topk_ids, topk_w, T, k, E, R, workspace, send_counts, send_offsets,
+                                              slot_send_row, ret_row, row_token, row_ids, row_w);
+  return cuda_status(moe::launch_ep_plan(a, s), "moe_ep_plan");
+}
+
+moe_status moe_ep_plan_host(const int32_t* topk_ids, const float* topk_w, int T, int k, int E, int R,
+                            int32_t* send_counts, int32_t* send_offsets, int32_t* slot_send_row, int32_t* ret_row,
+                            int32_t* row_token, int32_t* row_ids, float* row_w) {
+  moe_status st = check_ep_plan(topk_ids, topk_w, T, k, E, R, send_counts, send_offsets, slot_send_row, ret_row,
+                                row_token, row_ids, row_w);
+  if (st != MOE_OK) return st;
+  if (!moe::ep_plan_host(topk_ids, topk_w, T, k, E, R, send_counts, send_offsets, slot_send_row, ret_row, row_token,
+                         row_ids, row_w))
+    return fail(MOE_ERR_DEVICE, "moe_ep_plan_host: expert ids outside [0, E) were dropped");
+  return MOE_OK;
+}
+
+moe_status moe_ep_exchange_offsets(const int32_t* counts, int R, int rank, int32_t* dst_base, int32_t* recv_base,
+                                   int32_t* ret_base) {
+  MOE_REQUIRE(R >= 1 && R <= moe::kEpMaxRanks, "R must be in [1, 64]");
+  MOE_REQUIRE(rank >= 0 && rank < R, "rank must be in [0, R)");
+  MOE_REQUIRE(counts != nullptr && dst_base != nullptr && recv_base != nullptr && ret_base != nullptr,
+              "moe_ep_exchange_offsets: host arrays must not be NULL");
+  for (int i = 0; i < R * R; ++i) MOE_REQUIRE(counts[i] >= 0, "counts must be >= 0");
+  moe::ep_exchange_offsets_host(counts, R, rank, dst_base, recv_base, ret_base);
+  return MOE_OK;
+}
+
+moe_status moe_ep_pack(const void* x, int dtype, int T, int H, int k, int R, const int32_t* send_offsets,
+                       const int32_t* dst_base, const int32_t* row_token, const int32_t* row_ids, const float* row_w,
+                       void* const* dst_x, int32_t* const* dst_ids, float* const* dst_w, const int32_t* dst_cap,
+                       void* stream) {
+  const size_t es = dtype_size(dtype);
+  MOE_REQUIRE(es != 0, "dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(T >= 0, "T must be >= 0");
+  MOE_REQUIRE(H >= 1 && (H * es) % 16 == 0, "H * sizeof(dtype) must be a positive multiple of 16");
+  MOE_REQUIRE(k >= 1 && k <= 8, "k must be in [1, 8]");
+  MOE_REQUIRE(R >= 1 && R <= moe::kEpMaxRanks, "R must be in [1, 64]");
+  MOE_REQUIRE((long long)T * k < (1LL << 31), "T * k must be < 2^31");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE_PTR(x, 16, "x");
+  MOE_REQUIRE_PTR(send_offsets, 4, "send_offsets");
+  MOE_REQUIRE_PTR(dst_base, 4, "dst_base");
+  MOE_REQUIRE_PTR(row_token, 4, "row_token");
+  MOE_REQUIRE_PTR(row_ids, 4, "row_ids");
+  MOE_REQUIRE_PTR(row_w, 4, "row_w");
+  MOE_REQUIRE(dst_x != nullptr && dst_ids != nullptr && dst_w != nullptr && dst_cap != nullptr,
+              "dst_x, dst_ids, dst_w and dst_cap (host arrays of R entries) must not be NULL");
+  moe::EpDest dst = {};
+  for (int d = 0; d < R; ++d) {
+    MOE_REQUIRE(dst_cap[d] >= 0, "dst_cap entries must be >= 0");
+    if (dst_cap[d] > 0) {
+      MOE_REQUIRE_PTR(dst_x[d], 16, "dst_x[" + std::to_string(d) + "]");
+      MOE_REQUIRE_PTR(dst_ids[d], 4, "dst_ids[" + std::to_string(d) + "]");
+      MOE_REQUIRE_PTR(dst_w[d], 4, "dst_w[" + std::to_string(d) + "]");
+    }
+    dst.x[d] = dst_x[d];
+    dst.ids[d] = dst_ids[d];
+    dst.w[d] = dst_w[d];
+    dst.cap[d] = dst_cap[d];
+  }
+  const int max_rows = T * (k < R ? k : R);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err;
+  if (dtype == MOE_BF16)
+    err = moe::launch_ep_pack((const __nv_bfloat16*)x, T, H, k, R, max_rows, send_offsets, dst_base, row_token, row_ids,
+                              row_w, dst, s);
+  else
+    err = moe::launch_ep_pack((const float*)x, T, H, k, R, max_rows, send_offsets, dst_base, row_token, row_ids, row_w,
+                              dst, s);
+  return cuda_status(err, "moe_ep_pack");
+}
+
+moe_status moe_ep_recv_index(const int32_t* recv_ids, int T_recv, int k, int EL, int32_t* expert_counts,
+                             int32_t* expert_offsets, int32_t* slot_to_row, int32_t* row_to_slot, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  MOE_REQUIRE(T_recv >= 0, "T_recv must be >= 0");
+  moe_status st = check_k_e(k, EL);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE((long long)T_recv * k < (1LL << 31), "T_recv * k must be < 2^31");
+  MOE_REQUIRE_PTR(expert_counts, 4, "expert_counts");
+  MOE_REQUIRE_PTR(expert_offsets, 4, "expert_offsets");
+  MOE_REQUIRE_PTR(workspace, 16, "workspace");
+  const moe::DispatchGeom g = moe::make_dispatch_geom(T_recv, k, EL, 1);
+  MOE_REQUIRE(workspace_bytes >= moe::dispatch_ws_bytes(g), "workspace_bytes smaller than moe_dispatch_workspace_bytes(T_recv, k, EL, 1)");
+  if (T_recv > 0) {
+    MOE_REQUIRE_PTR(recv_ids, 4, "recv_ids");
+    MOE_REQUIRE_PTR(slot_to_row, 4, "slot_to_row");
+    MOE_REQUIRE_PTR(row_to_slot, 4, "row_to_slot");
+  }
+  // the one-rank dispatch of the received rows, index only (no row width: H is unused), no rank
+  // totals; -1 ids are padding
+  return cuda_status(moe::launch_dispatch<__nv_bfloat16>(g, 8, nullptr, recv_ids, workspace, nullptr, expert_counts,
+                                                         expert_offsets, nullptr, nullptr, slot_to_row, row_to_slot,
+                                                         nullptr, (cudaStream_t)stream, moe::kGridBarrierLimitNs, true),
+                     "moe_ep_recv_index");
 }
 
 moe_status moe_eplb_plan(const int64_t* load, int E, int R, int slots_per_rank, int32_t* phys_to_logical,
