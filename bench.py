@@ -447,6 +447,71 @@ def run_ours(args, wl):
                   "timing": "events per kernel, L2 flushed before each, median of the steps"}
         del y_part, y_m
 
+    # The exchange between ranks (moe_ep_*), its R ranks emulated on this GPU with their own
+    # buffers (the step of ep_round_trip_one_gpu, phase by phase): every rank's plan, the counts
+    # exchange (a host copy, outside the events), every rank's pack into the others' receive
+    # buffers, every rank's local experts over what it received, the partials' return and every
+    # rank's sum.  L2 flushed before the plan.  Its pack would cross NVLink on R GPUs.
+    ep_info = None
+    ep_bytes = wl.R * (wl.T // max(wl.R, 1)) * wl.k * (wl.H + wl.I) * (2 if wl.dtype == "bf16" else 4) * wl.R
+    if 1 < wl.R <= 64 and wl.T % wl.R == 0 and ep_bytes < (8 << 30):
+        from token_dispatch_combine_b200 import MoEEPRank
+        q = wl.T // wl.R
+        ranks = [MoEEPRank(r, wl.R, q, wl.H, wl.I, wl.E, wl.k, dt, device=dev, recv_capacity=wl.T)
+                 for r in range(wl.R)]
+        xs = [x[r * q:(r + 1) * q] for r in range(wl.R)]
+        lgs = [logits[r * q:(r + 1) * q].contiguous() for r in range(wl.R)]
+        EL = wl.E // wl.R
+        wsl = [(wg[d * EL:(d + 1) * EL], wu[d * EL:(d + 1) * EL], wd[d * EL:(d + 1) * EL]) for d in range(wl.R)]
+        phases = np.zeros(5)
+        n_ep = max(3, min(args.steps, 10))
+        for it in range(n_ep + 1):  # the first is a warm-up
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+            flush_and_hold()
+            ev[0].record(stream)
+            for r_, lg_ in zip(ranks, lgs):
+                r_.route_and_plan(lg_)
+            ev[1].record(stream)
+            counts = torch.stack([r_.plan.send_counts for r_ in ranks]).cpu().numpy()
+            for r_ in ranks:
+                r_.set_counts(counts)
+            # after that host round trip the GPU would wait for each launch of the host: hold it
+            # (~6 ms) while the host enqueues the rest, so the phase events measure GPU time
+            torch.cuda._sleep(HOLD_CYCLES * 30)
+            ev[2].record(stream)
+            for r_, x_ in zip(ranks, xs):
+                r_.pack_to(x_, ranks)
+            ev[3].record(stream)
+            for r_, w_ in zip(ranks, wsl):
+                r_.experts(*w_)
+            ev[4].record(stream)
+            for r_ in ranks:
+                r_.return_to(ranks)
+            ev[5].record(stream)
+            for r_ in ranks:
+                r_.finish()
+            ev[6].record(stream)
+            torch.cuda.synchronize()
+            if it:
+                phases += [ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3]), ev[3].elapsed_time(ev[4]),
+                           ev[4].elapsed_time(ev[5]), ev[5].elapsed_time(ev[6])]
+        phases /= n_ep
+        st, bits = moe_get_error()
+        if st != 0:
+            raise RuntimeError(f"device error word {bits} in the exchange between ranks")
+        rows = int(counts.sum())
+        b_ = 2 if wl.dtype == "bf16" else 4
+        pack_bytes = rows * (2 * wl.H * b_ + 16 * wl.k)
+        ep_info = {"ranks": wl.R, "tokens_per_rank": q, "rows_sent": rows, "slots": wl.S,
+                   "plan_us": phases[0] * 1e3, "pack_us": phases[1] * 1e3, "experts_us": phases[2] * 1e3,
+                   "return_us": phases[3] * 1e3, "finish_us": phases[4] * 1e3,
+                   "pack_gbs": pack_bytes / (phases[1] * 1e-3) / 1e9,
+                   "timing": "all R ranks on this GPU, events per phase summed over the ranks, L2 flushed "
+                             "before the plan; counts exchanged through the host outside the events, then the "
+                             "GPU held while the host enqueues the later phases; pack bytes = rows sent x (read "
+                             "+ write of a row) + ids/weights"}
+        del ranks
+
     # The router affinities fused with the top-k (moe_router_topk): logits = x W_r^T + bias on
     # tensor cores, then route's selection; L2 flushed before each call.  Not part of the step
     # above, which starts from given logits.
@@ -560,6 +625,26 @@ def run_ours(args, wl):
     barrier(world)
     e2e_ms = e_start.elapsed_time(e_end) / args.steps
     (e2e_ms,) = max_over_ranks([e2e_ms], world)
+    # One batch at a time, host in and host out on one stream (no overlap between batches): the
+    # latency of a single call sequence through the public API (upload x and logits from pinned
+    # memory, the step, download y).
+    x_dev1 = torch.empty_like(x)
+    l_dev1 = torch.empty_like(logits)
+    y_dev1 = torch.empty((wl.T, wl.H), dtype=dt, device=dev)
+    lat = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        x_dev1.copy_(x_h.view(dt) if dt == torch.bfloat16 else x_h, non_blocking=True)
+        l_dev1.copy_(l_h, non_blocking=True)
+        rt.forward(x_dev1, l_dev1, wg, wu, wd, y=y_dev1)
+        y_h.copy_(y_dev1.view(y_h.dtype) if y_h.dtype != dt else y_dev1, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            lat.append(a.elapsed_time(b))
+    (single_ms,) = max_over_ranks([statistics.median(lat)], world)
     st, bits = moe_get_error()
     if st != 0:
         raise RuntimeError(f"device error word {bits} during timing")
@@ -643,6 +728,7 @@ def run_ours(args, wl):
                                       "events per call; bytes T*H*2 + E*H*2 + T*k*8"}),
             **({} if eplb is None else {"eplb": eplb}),
             **({} if masked is None else {"masking_form": masked}),
+            **({} if ep_info is None else {"exchange_between_ranks_one_gpu": ep_info}),
             "graph_replay_ms": graph_ms,
             **({} if graph_err is None else {"graph_replay_error": graph_err}),
             "ffn_tiling": {"gate_up": "pair" if tiling == FFN_TILING_PAIR else "single",
@@ -661,7 +747,10 @@ def run_ours(args, wl):
         },
         "e2e": {"value": wl.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_np.nbytes + logits_np.nbytes), "d2h_bytes_per_step": int(y_h.numel() * y_h.element_size()),
-                "api": "MoEHostPipeline (upload, compute and download of consecutive steps overlap)"},
+                "api": "MoEHostPipeline (upload, compute and download of consecutive steps overlap)",
+                "single_batch_ms": single_ms,
+                "single_batch": "one batch host to host on one stream (upload x and logits, MoERoundTrip.forward, "
+                                "download y), no overlap with other batches; median of the steps"},
         "gpu_launches": MoERoundTrip.KERNELS_PER_FORWARD * args.steps,  # kernels of this library in the timed region
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

@@ -52,6 +52,20 @@ def test_workspace_query_is_host_only():
     assert lib.moe_dispatch_workspace_bytes(-1, 4, 32, 8) == 0
 
 
+def test_counted_pair_workspace_query_is_host_only():
+    """The counted pair counts in chunks of at most 128 slots (moe_dispatch: 512), so its
+    workspace holds at least as many chunk counts; both queries reject bad sizes with 0."""
+    lib = _native.lib()
+    for T, k, E, R in [(4096, 4, 32, 8), (128, 8, 256, 32), (8192, 8, 256, 32), (1, 1, 4, 2), (1000, 3, 6, 1)]:
+        plain = lib.moe_dispatch_workspace_bytes(T, k, E, R)
+        counted = lib.moe_route_count_workspace_bytes(T, k, E, R)
+        assert counted >= plain > 0
+    # GPT-OSS shape: 8 ranks x 2048 slots, 512-slot chunks -> 32 chunks; 128-slot chunks -> 128
+    assert lib.moe_dispatch_workspace_bytes(4096, 4, 32, 8) == 256 + 4 * (2 * 32 * 32 + 16384 + 32)
+    assert lib.moe_route_count_workspace_bytes(4096, 4, 32, 8) == 256 + 4 * (2 * 128 * 32 + 16384 + 32)
+    assert lib.moe_route_count_workspace_bytes(-1, 4, 32, 8) == 0
+
+
 FAKE = 0x1000  # never dereferenced: every call below fails validation first
 
 
@@ -112,6 +126,18 @@ def test_dispatch_timeout_selftest_rejects(limit_us, T, needle):
                                            None, FAKE, 1 << 20, limit_us, None)
     assert st == _native.MOE_ERR_INVALID_ARG
     assert needle in lib.moe_last_error_message()
+
+
+def test_route_count_rejects_a_workspace_sized_for_moe_dispatch():
+    lib = _native.lib()
+    T, k, E, R = 4096, 4, 32, 8
+    small = lib.moe_dispatch_workspace_bytes(T, k, E, R)
+    assert lib.moe_route_count(FAKE, T, E, k, R, FAKE, FAKE, FAKE, small, None) == _native.MOE_ERR_INVALID_ARG
+    assert b"moe_route_count_workspace_bytes" in lib.moe_last_error_message()
+    st = lib.moe_dispatch_counted(FAKE, 1, T, 64, FAKE, k, E, R, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                  small, None)
+    assert st == _native.MOE_ERR_INVALID_ARG
+    assert b"moe_route_count_workspace_bytes" in lib.moe_last_error_message()
 
 
 @pytest.mark.parametrize("kw,needle", [

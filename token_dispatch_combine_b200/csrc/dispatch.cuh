@@ -9,7 +9,8 @@
 // [r*E/R, (r+1)*E/R), so the expert-major row order is rank-major.
 //
 // One cooperative launch (every CTA resident at once), three phases split by
-// one or two bounded grid barriers:
+// one or two bounded grid barriers (a counted dispatch with a small count
+// table has none, and is launched plainly):
 //  1. per chunk of <= 512 slots (chunks never straddle a source rank, token
 //     t's source rank being t*R/T): each slot's stable rank among the
 //     same-expert slots of its chunk, without atomics -- __match_any_sync
@@ -43,6 +44,12 @@
 namespace moe {
 
 constexpr int kDispatchThreads = 512;
+// CTAs of the dispatch kernel resident per SM: 2 caps it at 64 registers per
+// thread (no spills), twice the warps -- and the bytes in flight -- of the 84
+// registers it takes unbounded (one CTA per SM).
+#ifndef MOE_DISPATCH_MIN_BLOCKS
+#define MOE_DISPATCH_MIN_BLOCKS 2
+#endif
 constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kScatterVecsPerLane = 4;                   // 16-byte vectors in flight per lane
 constexpr int kScatterSlice = 32 * kScatterVecsPerLane;  // 16-byte vectors of a row per warp item
@@ -463,7 +470,7 @@ __device__ __forceinline__ void dispatch_phases(
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(
+__global__ void __launch_bounds__(kDispatchThreads, MOE_DISPATCH_MIN_BLOCKS) dispatch_kernel(
     DispatchGeom g, int H, int nslices, int tpc, const T* __restrict__ x, const int32_t* __restrict__ ids, DispatchWs ws,
     uint64_t limit_ns, int allow_pad, int counted, T* __restrict__ x_disp, int32_t* __restrict__ expert_counts,
     int32_t* __restrict__ expert_offsets, int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets,
@@ -619,13 +626,24 @@ cudaError_t launch_dispatch(const DispatchGeom& g, int H, const T* x, const int3
   cfg.blockDim = dim3(kDispatchThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
+  // A counted dispatch with a small count table never waits on a grid barrier,
+  // so it needs no co-residency: a plain launch lets its CTAs start as the
+  // previous kernel's SMs free up.  Every other form is a cooperative launch.
+  const bool grid_sync = !(counted && (size_t)g.nchunks * g.E <= kSmallCountTable);
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  int na = 0;
+  if (grid_sync) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+    ++na;
+  }
+  if (MOE_PDL) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = MOE_PDL ? 2 : 1;
+  cfg.numAttrs = na;
   err = cudaLaunchKernelEx(&cfg, kern, g, H, nslices, tpc, x, ids, ws, limit_ns, (int)allow_pad, (int)counted, x_disp,
                            expert_counts, expert_offsets, rank_counts, rank_offsets, slot_to_row, row_to_slot,
                            src_expert_counts);
