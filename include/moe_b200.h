@@ -455,7 +455,8 @@ moe_status moe_reduce_rank_partials(const void* y_part, int dtype, int T, int H,
  * moe_ep_recv_index: the received rows' counting sort by local expert:
  *   recv_ids       [T_recv, k]  received row_ids (-1 = padding, never
  *                               flagged; rows past the received count must
- *                               be all -1)
+ *                               be all -1); k may exceed EL (a row holds at
+ *                               most min(k, EL) local ids)
  *   expert_counts  [EL], expert_offsets [EL + 1]  out
  *   slot_to_row    [T_recv * k] out: GEMM row of (received row q, choice i),
  *                               -1 for padding

@@ -118,6 +118,17 @@ def test_noalloc_dispatch_rejects_bad_arguments_before_any_device_work():
     assert b"slot_to_row" in lib.moe_last_error_message()
 
 
+def test_ep_recv_index_accepts_more_columns_than_local_experts():
+    """A received row holds at most min(k, E/R) local ids padded to k columns: k > E/R is valid
+    (rejected here only for the missing workspace size, i.e. after the k / EL checks)."""
+    lib = _native.lib()
+    st = lib.moe_ep_recv_index(FAKE, 10, 8, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None)
+    assert st == _native.MOE_ERR_INVALID_ARG
+    assert b"workspace_bytes" in lib.moe_last_error_message()
+    assert lib.moe_ep_recv_index(FAKE, 10, 9, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert b"k must" in lib.moe_last_error_message()
+
+
 @pytest.mark.parametrize("limit_us,T,needle", [(0, 8, b"limit_us"), (2000000, 8, b"limit_us"), (20, 0, b"T must"),
                                                (20, -3, b"T must")])
 def test_dispatch_timeout_selftest_rejects(limit_us, T, needle):

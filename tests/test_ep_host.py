@@ -37,7 +37,7 @@ def _routing(T, E, k, seed, hot=0.0, R=1):
 
 @pytest.mark.parametrize("T,E,k,R,hot", [(300, 16, 4, 4, 0.0), (257, 32, 8, 8, 1.0), (64, 8, 1, 2, 0.0),
                                          (1000, 256, 8, 32, 0.5), (50, 6, 6, 3, 0.0), (40, 4, 2, 1, 0.0),
-                                         (0, 8, 2, 2, 0.0), (2500, 64, 8, 64, 0.0)])
+                                         (0, 8, 2, 2, 0.0), (2500, 64, 8, 64, 0.0), (500, 8, 4, 4, 0.0)])
 def test_host_plan_matches_oracle(T, E, k, R, hot):
     ids, w = _routing(T, E, k, T + E, hot, R)
     got = moe_ep_plan_host(ids, w, E, R)

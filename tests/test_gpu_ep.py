@@ -78,6 +78,7 @@ def _split(layer, sizes):
     ("bf16", (200, 0, 150, 300)),
     ("f32", (60, 41)),
     ("bf16_e256", (96, 96, 31, 1, 64, 0, 12, 100)),
+    ("bf16_el2", (100, 50, 0, 80)),  # 2 experts per rank, top-4: rows carry at most 2 of 4 id columns
 ])
 def test_round_trip_of_ranks_on_one_gpu(name, sizes):
     from token_dispatch_combine_b200 import ep_round_trip_one_gpu, moe_get_error
@@ -86,7 +87,8 @@ def test_round_trip_of_ranks_on_one_gpu(name, sizes):
     R = len(sizes)
     wl = {"bf16": W("ep_bf16", T=T, H=256, I=384, E=16, k=4, R=R, dtype="bf16", seed=41, bias="zipf1.2"),
           "f32": W("ep_f32", T=T, H=96, I=160, E=8, k=3, R=R, dtype="f32", seed=42),
-          "bf16_e256": W("ep_e256", T=T, H=128, I=128, E=256, k=8, R=R, dtype="bf16", seed=43, bias="normal0.5")}[name]
+          "bf16_e256": W("ep_e256", T=T, H=128, I=128, E=256, k=8, R=R, dtype="bf16", seed=43, bias="normal0.5"),
+          "bf16_el2": W("ep_el2", T=T, H=128, I=192, E=8, k=4, R=R, dtype="bf16", seed=44)}[name]
     layer = DeviceLayer(wl)
     start, xs, lg = _split(layer, sizes)
     ranks = _ranks(sizes, wl, layer.x_dev.dtype)

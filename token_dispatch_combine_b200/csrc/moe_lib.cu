@@ -729,8 +729,9 @@ moe_status moe_ep_recv_index(const int32_t* recv_ids, int T_recv, int k, int EL,
                              int32_t* expert_offsets, int32_t* slot_to_row, int32_t* row_to_slot, void* workspace,
                              size_t workspace_bytes, void* stream) {
   MOE_REQUIRE(T_recv >= 0, "T_recv must be >= 0");
-  moe_status st = check_k_e(k, EL);
-  if (st != MOE_OK) return st;
+  // a received row holds at most min(k, EL) local ids, padded with -1 to k columns: k may exceed EL
+  MOE_REQUIRE(EL >= 1 && EL <= 1024, "EL must be in [1, 1024]");
+  MOE_REQUIRE(k >= 1 && k <= 8, "k must be in [1, 8]");
   MOE_REQUIRE((long long)T_recv * k < (1LL << 31), "T_recv * k must be < 2^31");
   MOE_REQUIRE_PTR(expert_counts, 4, "expert_counts");
   MOE_REQUIRE_PTR(expert_offsets, 4, "expert_offsets");
