@@ -23,7 +23,13 @@ The step of one rank (``MoEEPRank``):
   finish    each token's partials summed: its output.
 ``ep_round_trip_one_gpu`` runs R ranks on one GPU, the exchange through
 device memory (each rank's pack writes straight into the other ranks'
-receive buffers, as peer stores would).
+receive buffers, as peer stores would).  ``ep_share_buffers`` +
+``ep_round_trip_ranks`` run it with one process per rank: every rank's
+receive and return buffers are mapped into every other rank's process (CUDA
+IPC, one node), so the pack kernel stores rows straight into the peers'
+memory and the partials return by peer copies; the counts go through
+``torch.distributed`` and host barriers separate the phases, so no kernel
+ever waits on another rank's kernel.
 """
 from __future__ import annotations
 
@@ -270,3 +276,63 @@ def ep_round_trip_one_gpu(ranks, xs, logits, w_gate, w_up, w_down, stream=None):
     for r in ranks:
         r.return_to(ranks, stream)
     return [r.finish(stream) for r in ranks[:R]]
+
+
+class EpPeer:
+    """Another rank's receive buffers (x_recv, recv_ids, recv_w) and return buffer (y_ret) as
+    mapped into this process: what ``MoEEPRank.pack_to`` and ``return_to`` write into."""
+
+    def __init__(self, rank, x_recv, recv_ids, recv_w, y_ret):
+        self.rank = rank
+        self.x_recv, self.recv_ids, self.recv_w, self.y_ret = x_recv, recv_ids, recv_w, y_ret
+
+
+def ep_share_buffers(me: MoEEPRank, group=None) -> list:
+    """Every rank's buffers as seen from this process (one process per rank, all on one node):
+    this rank's own ``MoEEPRank`` at its index, an ``EpPeer`` for each other rank.  The buffers'
+    CUDA IPC handles (torch's tensor sharing) travel through ``all_gather_object`` on ``group``;
+    opening one maps the owner's memory (with peer access when it lives on another GPU).  The
+    owners must keep their ``MoEEPRank`` alive while any peer holds the mapping."""
+    import io
+    import pickle
+    from multiprocessing.reduction import ForkingPickler
+
+    import torch.distributed as dist
+    import torch.multiprocessing  # noqa: F401  (registers the CUDA tensor reductions)
+    def handles_for_one_peer():  # torch counts each pickled handle as one receiver
+        buf = io.BytesIO()
+        ForkingPickler(buf, pickle.HIGHEST_PROTOCOL).dump((me.x_recv, me.recv_ids, me.recv_w, me.y_ret))
+        return buf.getvalue()
+
+    mine = [b"" if d == me.rank else handles_for_one_peer() for d in range(me.R)]
+    every = [None] * me.R
+    dist.all_gather_object(every, mine, group=group)  # every[s][d]: source s's handles for rank d
+    return [me if s == me.rank else EpPeer(s, *pickle.loads(every[s][me.rank])) for s in range(me.R)]
+
+
+def ep_round_trip_ranks(me: MoEEPRank, peers: list, x, logits, w_gate, w_up, w_down, group=None):
+    """One step of the expert-parallel layer for this process's rank, the other ranks running the
+    same call in their processes.  ``peers`` from ``ep_share_buffers``; w_* this rank's E/R local
+    experts ([EL, H, I] / [EL, I, H]).  Phases (each ends with this rank's kernels done and a
+    barrier of all ranks, so a rank writes into a peer's buffer only once the peer has finished
+    with it): plan and counts exchange; pack into the destinations' receive buffers; local
+    experts and return of the partials into the sources' return buffers; then the sum of each
+    token's partials, which is returned."""
+    import torch.distributed as dist
+
+    def fence():
+        torch.cuda.synchronize(me.device)
+        dist.barrier(group=group)
+
+    me.route_and_plan(logits)
+    counts = [None] * me.R
+    dist.all_gather_object(counts, me.plan.send_counts.cpu().numpy().astype(np.int32), group=group)
+    me.set_counts(np.stack(counts))
+    fence()  # every receive buffer is free (its owner finished the previous step with it)
+    me.pack_to(x, peers)
+    fence()  # every row has landed
+    me.experts(w_gate, w_up, w_down)
+    me.return_to(peers)
+    fence()  # every partial has returned
+    return me.finish()
+
