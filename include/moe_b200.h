@@ -464,6 +464,14 @@ moe_status moe_reduce_rank_partials(const void* y_part, int dtype, int T, int H,
  *   workspace      moe_dispatch_workspace_bytes(T_recv, k, EL, 1) bytes,
  *                  zero-filled once (as moe_dispatch's)
  * GEMM rows are ordered by (local expert, received row): stable.
+ *
+ * moe_enable_peer_access (host; enqueues nothing): lets kernels launched on
+ * the CURRENT device load and store memory that lives on device peer_device
+ * (a peer's receive buffers given to moe_ep_pack), i.e.
+ * cudaDeviceEnablePeerAccess from the current device.  peer_device equal to
+ * the current device, or access already enabled, is MOE_OK; a pair of
+ * devices without peer capability is MOE_ERR_UNSUPPORTED; peer_device < 0 or
+ * not below the device count is MOE_ERR_INVALID_ARG.
  */
 size_t moe_ep_plan_workspace_bytes(int T, int R);
 moe_status moe_ep_plan(const int32_t* topk_ids, const float* topk_w, int T, int k, int E, int R,
@@ -482,6 +490,7 @@ moe_status moe_ep_pack(const void* x, int dtype, int T, int H, int k, int R, con
 moe_status moe_ep_recv_index(const int32_t* recv_ids, int T_recv, int k, int EL, int32_t* expert_counts,
                              int32_t* expert_offsets, int32_t* slot_to_row, int32_t* row_to_slot, void* workspace,
                              size_t workspace_bytes, void* stream);
+moe_status moe_enable_peer_access(int peer_device);
 
 /*
  * Expert placement with replicas -- an expert-parallel load balancer:

@@ -279,3 +279,8 @@ def test_round_trip_gathers_where_the_ffn_streams_weights():
     assert rule(383 * 32 // 4, 4, 32, bf16)   # just under 384 rows per expert
     assert not rule(384 * 32 // 4, 4, 32, bf16)
     assert not rule(128, 8, 256, f32)         # float32 layers keep the row-moving dispatch
+
+
+def test_enable_peer_access_rejects_a_negative_device():
+    assert _native.lib().moe_enable_peer_access(-1) == _native.MOE_ERR_INVALID_ARG
+    assert b"peer_device" in _native.lib().moe_last_error_message()

@@ -158,3 +158,9 @@ def test_ranks_as_processes_exchange_through_ipc(sizes):
         if sizes[r]:
             whole, worst, _ = row_errors(got["y"][0], ep["y"][r])
             assert whole <= TOL["bf16"] and worst <= TOL["bf16"], (r, whole, worst)
+
+
+def test_enable_peer_access_on_one_gpu():
+    from token_dispatch_combine_b200 import _native, moe_enable_peer_access
+    moe_enable_peer_access(torch.cuda.current_device())  # the device itself: nothing to enable
+    assert _native.lib().moe_enable_peer_access(torch.cuda.device_count()) == _native.MOE_ERR_INVALID_ARG

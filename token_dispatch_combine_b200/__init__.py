@@ -15,8 +15,8 @@ from .api import (DispatchOut, EplbPlan, MoEBalancedRoundTrip, MoEHostPipeline, 
                   moe_ffn_tiling_for, moe_get_error, moe_get_ffn_tiling, moe_route, moe_router_topk,
                   moe_set_ffn_tiling, new_dispatch_workspace)
 from .ep import (EpPeer, EpPlan, MoEEPRank, ep_round_trip_one_gpu, ep_round_trip_ranks, ep_share_buffers,
-                 moe_ep_exchange_offsets, moe_ep_pack, moe_ep_plan, moe_ep_plan_host, moe_ep_plan_workspace_bytes,
-                 moe_ep_recv_index)
+                 moe_enable_peer_access, moe_ep_exchange_offsets, moe_ep_pack, moe_ep_plan, moe_ep_plan_host,
+                 moe_ep_plan_workspace_bytes, moe_ep_recv_index)
 from ._native import FFN_DOWN, FFN_GATE_UP, FFN_TILING_AUTO, FFN_TILING_PAIR, FFN_TILING_SINGLE, MoeError
 
 _native.lib()  # build (if needed) and load now: fail loudly at import
@@ -28,7 +28,7 @@ __all__ = [
     "moe_ffn_tiling_for", "FFN_TILING_AUTO", "FFN_TILING_SINGLE", "FFN_TILING_PAIR", "FFN_GATE_UP", "FFN_DOWN",
     "moe_router_topk", "EplbPlan", "MoEBalancedRoundTrip", "moe_eplb_plan", "moe_eplb_remap", "moe_eplb_replicate",
     "moe_combine_rank_partials", "moe_reduce_rank_partials", "EpPeer", "EpPlan", "MoEEPRank", "ep_round_trip_one_gpu",
-    "ep_round_trip_ranks", "ep_share_buffers",
+    "ep_round_trip_ranks", "ep_share_buffers", "moe_enable_peer_access",
     "moe_ep_exchange_offsets", "moe_ep_pack", "moe_ep_plan", "moe_ep_plan_host", "moe_ep_plan_workspace_bytes",
     "moe_ep_recv_index", "moe_route_count", "moe_dispatch_counted", "moe_ffn_down_combine", "moe_combine_finalize",
     "moe_route_count_workspace_bytes",

@@ -27,7 +27,7 @@ EXPORTS = (
     "moe_ffn_gate_up_gather", "moe_expert_ffn_gather", "moe_eplb_plan", "moe_eplb_remap", "moe_eplb_replicate",
     "moe_selftest_dispatch_timeout", "moe_combine_rank_partials", "moe_reduce_rank_partials",
     "moe_ep_plan_workspace_bytes", "moe_ep_plan", "moe_ep_plan_host", "moe_ep_exchange_offsets", "moe_ep_pack",
-    "moe_ep_recv_index", "moe_route_count", "moe_dispatch_counted", "moe_ffn_down_combine", "moe_combine_finalize",
+    "moe_enable_peer_access", "moe_ep_recv_index", "moe_route_count", "moe_dispatch_counted", "moe_ffn_down_combine", "moe_combine_finalize",
     "moe_route_count_workspace_bytes",
 )
 
@@ -72,6 +72,7 @@ def _configure(lib):
         "moe_ep_plan": ([vp, vp, i32, i32, i32, i32] + [vp] * 7 + [vp, sz, vp], i32),
         "moe_ep_plan_host": ([vp, vp, i32, i32, i32, i32] + [vp] * 7, i32),
         "moe_ep_exchange_offsets": ([vp, i32, i32, vp, vp, vp], i32),
+        "moe_enable_peer_access": ([i32], i32),
         "moe_ep_pack": ([vp, i32, i32, i32, i32, i32] + [vp] * 5 + [vp] * 4 + [vp], i32),
         "moe_ep_recv_index": ([vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp], i32),
         "moe_route_count_workspace_bytes": ([i32, i32, i32, i32], sz),

@@ -680,6 +680,27 @@ moe_status moe_ep_exchange_offsets(const int32_t* counts, int R, int rank, int32
   return MOE_OK;
 }
 
+moe_status moe_enable_peer_access(int peer_device) {
+  MOE_REQUIRE(peer_device >= 0, "peer_device must be >= 0");
+  int dev = 0, n = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_status(err, "cudaGetDevice");
+  err = cudaGetDeviceCount(&n);
+  if (err != cudaSuccess) return cuda_status(err, "cudaGetDeviceCount");
+  MOE_REQUIRE(peer_device < n, "peer_device must be below the device count");
+  if (peer_device == dev) return MOE_OK;
+  int can = 0;
+  err = cudaDeviceCanAccessPeer(&can, dev, peer_device);
+  if (err != cudaSuccess) return cuda_status(err, "cudaDeviceCanAccessPeer");
+  if (!can) return fail(MOE_ERR_UNSUPPORTED, "the current device cannot access peer_device's memory");
+  err = cudaDeviceEnablePeerAccess(peer_device, 0);
+  if (err == cudaErrorPeerAccessAlreadyEnabled) {
+    (void)cudaGetLastError();  // clear the (non-sticky) error this call recorded
+    return MOE_OK;
+  }
+  return cuda_status(err, "cudaDeviceEnablePeerAccess");
+}
+
 moe_status moe_ep_pack(const void* x, int dtype, int T, int H, int k, int R, const int32_t* send_offsets,
                        const int32_t* dst_base, const int32_t* row_token, const int32_t* row_ids, const float* row_w,
                        void* const* dst_x, int32_t* const* dst_ids, float* const* dst_w, const int32_t* dst_cap,

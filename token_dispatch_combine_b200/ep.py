@@ -161,6 +161,12 @@ def moe_ep_recv_index(recv_ids, EL: int, expert_counts, expert_offsets, slot_to_
         _stream(stream)), "moe_ep_recv_index")
 
 
+def moe_enable_peer_access(peer_device: int) -> None:
+    """Let kernels on the current device load and store memory of device ``peer_device``
+    (no-op for the current device itself or when already enabled)."""
+    check(_native.lib().moe_enable_peer_access(int(peer_device)), "moe_enable_peer_access")
+
+
 class MoEEPRank:
     """One rank of an expert-parallel MoE layer over R ranks: its T tokens, its E/R local
     experts, and every buffer of its step (allocated here, once).  ``recv_capacity`` bounds
@@ -307,7 +313,12 @@ def ep_share_buffers(me: MoEEPRank, group=None) -> list:
     mine = [b"" if d == me.rank else handles_for_one_peer() for d in range(me.R)]
     every = [None] * me.R
     dist.all_gather_object(every, mine, group=group)  # every[s][d]: source s's handles for rank d
-    return [me if s == me.rank else EpPeer(s, *pickle.loads(every[s][me.rank])) for s in range(me.R)]
+    peers = [me if s == me.rank else EpPeer(s, *pickle.loads(every[s][me.rank])) for s in range(me.R)]
+    with torch.cuda.device(me.device):
+        for p in peers:  # the pack kernel stores into peers' buffers that may live on other GPUs
+            if p.x_recv.device != me.device:
+                moe_enable_peer_access(p.x_recv.device.index)
+    return peers
 
 
 def ep_round_trip_ranks(me: MoEEPRank, peers: list, x, logits, w_gate, w_up, w_down, group=None):
