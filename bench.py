@@ -610,21 +610,40 @@ def run_ours(args, wl):
     x_h = torch.from_numpy(x_np.view(np.int16) if x_np.dtype == np.uint16 else x_np).pin_memory()
     l_h = torch.from_numpy(logits_np).pin_memory()
     y_h = torch.empty((wl.T, wl.H), dtype=torch.int16 if dt == torch.bfloat16 else torch.float32).pin_memory()
-    pipe = MoEHostPipeline(rt, wg, wu, wd, compute_stream=stream)
+    pipe = MoEHostPipeline(rt, wg, wu, wd, compute_stream=stream, graphs=args.e2e_graphs == "on")
     pipe.run([(x_h, l_h, y_h)] * max(1, args.warmup))
     torch.cuda.synchronize()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     torch.cuda._sleep(HOLD_CYCLES * 10)  # let the host enqueue ahead of the GPU
-    e_start.record(stream)
-    pipe.h2d.wait_stream(stream)
-    pipe.run([(x_h, l_h, y_h)] * args.steps)
-    e_end.record(pipe.d2h)
-    torch.cuda.synchronize()
+    with ClockSampler(local) as e2e_clocks:
+        e_start.record(stream)
+        pipe.h2d.wait_stream(stream)
+        h0 = time.perf_counter()
+        pipe.run([(x_h, l_h, y_h)] * args.steps)
+        host_enqueue_ms = (time.perf_counter() - h0) * 1e3 / args.steps  # the host's time to enqueue a step
+        e_end.record(pipe.d2h)
+        torch.cuda.synchronize()
     barrier(world)
     e2e_ms = e_start.elapsed_time(e_end) / args.steps
     (e2e_ms,) = max_over_ranks([e2e_ms], world)
+    # The same steps back to back without the copies (graph replays on the device buffers, no L2
+    # flush or hold between steps): what the pipeline's compute alone sustains.
+    b2b_ms = None
+    if pipe.graphs is not None:
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda._sleep(HOLD_CYCLES * 10)
+        g_start, g_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g_start.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                pipe.graphs[0].replay()
+        g_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        (b2b_ms,) = max_over_ranks([g_start.elapsed_time(g_end) / args.steps], world)
     # One batch at a time, host in and host out on one stream (no overlap between batches): the
     # latency of a single call sequence through the public API (upload x and logits from pinned
     # memory, the step, download y).
@@ -747,7 +766,13 @@ def run_ours(args, wl):
         },
         "e2e": {"value": wl.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_np.nbytes + logits_np.nbytes), "d2h_bytes_per_step": int(y_h.numel() * y_h.element_size()),
-                "api": "MoEHostPipeline (upload, compute and download of consecutive steps overlap)",
+                "api": "MoEHostPipeline (upload, compute and download of consecutive steps overlap"
+                       + ("; each step one CUDA graph replay)" if args.e2e_graphs == "on" else "; eager calls)"),
+                "host_enqueue_ms_per_step": host_enqueue_ms,
+                "compute_back_to_back_ms": b2b_ms,
+                "compute_back_to_back": "the same steps' graph replays back to back with no copies, no L2 flush "
+                                        "and no hold between them",
+                "clocks": e2e_clocks.summary(),
                 "single_batch_ms": single_ms,
                 "single_batch": "one batch host to host on one stream (upload x and logits, MoERoundTrip.forward, "
                                 "download y), no overlap with other batches; median of the steps"},
@@ -778,6 +803,8 @@ def main():
     ap.add_argument("--combine-in-down", default="off", choices=["on", "off"],
                     help="on: the down projection's epilogue does the combine (moe_ffn_down_combine, float32 "
                          "atomics into a [T, H] accumulator) and a finalize kernel rounds it into y")
+    ap.add_argument("--e2e-graphs", default="on", choices=["on", "off"],
+                    help="on: the end-to-end pipeline replays one captured CUDA graph per step")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false",
                     help="skip the CPU oracle leg (used for profiler runs)")
     args = ap.parse_args()

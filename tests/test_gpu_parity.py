@@ -236,9 +236,10 @@ def test_identity_experts_combine_reproduces_input():
     np.testing.assert_allclose(dev_to_np(y), layer.x, rtol=0, atol=1e-6 * np.abs(layer.x).max())
 
 
-def test_host_pipeline_matches_forward():
-    """MoEHostPipeline (overlapped upload/compute/download) gives, per batch, exactly
-    what a plain forward of that batch gives."""
+@pytest.mark.parametrize("graphs", [True, False])
+def test_host_pipeline_matches_forward(graphs):
+    """MoEHostPipeline (overlapped upload/compute/download; each batch a CUDA graph replay,
+    or eager calls) gives, per batch, exactly what a plain forward of that batch gives."""
     from token_dispatch_combine_b200 import MoEHostPipeline, MoERoundTrip
     wl = W("pipe", T=300, H=256, I=384, E=8, k=2, R=4, dtype="bf16", seed=19)
     layer = DeviceLayer(wl)
@@ -251,7 +252,7 @@ def test_host_pipeline_matches_forward():
         batches.append((x.view(torch.int16).cpu().pin_memory(), lg.cpu().pin_memory(),
                         torch.empty(wl.T, wl.H, dtype=torch.int16).pin_memory()))
     torch.cuda.synchronize()
-    pipe = MoEHostPipeline(rt, layer.w_gate, layer.w_up, layer.w_down)
+    pipe = MoEHostPipeline(rt, layer.w_gate, layer.w_up, layer.w_down, graphs=graphs)
     pipe.run(batches).synchronize()
     torch.cuda.synchronize()
     for (_, _, yh), y in zip(batches, want):

@@ -545,22 +545,32 @@ class MoEHostPipeline:
     y ends there.  Three CUDA streams overlap the host->device copy of batch
     i+1 and the device->host copy of batch i-1 with the compute of batch i;
     device inputs and outputs are double-buffered, and events order every
-    reuse of a buffer after the work that last touched it.
+    reuse of a buffer after the work that last touched it.  With ``graphs``
+    (the default) the round trip of each buffer set is a captured CUDA graph,
+    replayed once per batch.
     """
 
-    def __init__(self, rt: MoERoundTrip, w_gate, w_up, w_down, compute_stream=None):
+    def __init__(self, rt: MoERoundTrip, w_gate, w_up, w_down, compute_stream=None, graphs=True):
         self.rt = rt
         self.w = (w_gate, w_up, w_down)
         dev = rt.device
         self.comp = compute_stream if compute_stream is not None else torch.cuda.current_stream(dev)
         self.h2d = torch.cuda.Stream(dev)
         self.d2h = torch.cuda.Stream(dev)
-        self.x_dev = [torch.empty((rt.T, rt.H), dtype=rt.dtype, device=dev) for _ in range(2)]
-        self.l_dev = [torch.empty((rt.T, rt.E), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.x_dev = [torch.zeros((rt.T, rt.H), dtype=rt.dtype, device=dev) for _ in range(2)]
+        self.l_dev = [torch.zeros((rt.T, rt.E), dtype=torch.float32, device=dev) for _ in range(2)]
         self.y_dev = [torch.empty((rt.T, rt.H), dtype=rt.dtype, device=dev) for _ in range(2)]
         ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
         self.in_ready, self.in_free, self.out_ready, self.out_free = ev(), ev(), ev(), ev()
         self._used = [False, False]
+        self.graphs = None
+        if graphs:
+            # one CUDA graph per buffer set: a step then costs the host one launch instead of the
+            # round trip's calls (first use of each kernel happens here, outside the capture)
+            rt.forward(self.x_dev[0], self.l_dev[0], *self.w, stream=self.comp, y=self.y_dev[0])
+            self.comp.synchronize()
+            self.graphs = [rt.capture(self.x_dev[b], self.l_dev[b], *self.w, y=self.y_dev[b]) for b in range(2)]
+            torch.cuda.synchronize(dev)
 
     @staticmethod
     def _as_dev_dtype(host: torch.Tensor, dev: torch.Tensor) -> torch.Tensor:
@@ -581,7 +591,11 @@ class MoEHostPipeline:
             self.comp.wait_event(self.in_ready[b])
             if self._used[b]:
                 self.comp.wait_event(self.out_free[b])  # y of batch i-2 has been copied out
-            self.rt.forward(self.x_dev[b], self.l_dev[b], *self.w, stream=self.comp, y=self.y_dev[b])
+            if self.graphs is not None:
+                with torch.cuda.stream(self.comp):
+                    self.graphs[b].replay()
+            else:
+                self.rt.forward(self.x_dev[b], self.l_dev[b], *self.w, stream=self.comp, y=self.y_dev[b])
             self.in_free[b].record(self.comp)
             self.out_ready[b].record(self.comp)
             self.d2h.wait_event(self.out_ready[b])
