@@ -305,6 +305,7 @@ def ep_share_buffers(me: MoEEPRank, group=None) -> list:
 
     import torch.distributed as dist
     import torch.multiprocessing  # noqa: F401  (registers the CUDA tensor reductions)
+
     def handles_for_one_peer():  # torch counts each pickled handle as one receiver
         buf = io.BytesIO()
         ForkingPickler(buf, pickle.HIGHEST_PROTOCOL).dump((me.x_recv, me.recv_ids, me.recv_w, me.y_ret))
