@@ -35,7 +35,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 STEPS = 2
 
 
-def _workload(sizes):
+def _workload(name, sizes):
+    if name == "e256":  # DeepSeek-R1-like routing: 256 experts, top-8, 8 ranks of 32 experts
+        return synth.Workload("ep_ipc_e256", T=sum(sizes), H=128, I=128, E=256, k=8, R=len(sizes), dtype="bf16",
+                              seed=47, bias="normal0.5")
     return synth.Workload("ep_ipc", T=sum(sizes), H=256, I=384, E=16, k=4, R=len(sizes), dtype="bf16", seed=46,
                           bias="zipf1.2")
 
@@ -61,7 +64,7 @@ def _require_shared_gpu():
         pytest.skip(f"GPU compute mode {mode}: one process per GPU only")
 
 
-def _rank_worker(rank, sizes, port, q):
+def _rank_worker(rank, name, sizes, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -73,7 +76,7 @@ def _rank_worker(rank, sizes, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=R, timeout=datetime.timedelta(seconds=120))
     try:
         torch.cuda.set_device(0)
-        wl = _workload(sizes)
+        wl = _workload(name, sizes)
         layer = Layer(wl)
         start = np.concatenate([[0], np.cumsum(sizes)]).astype(int)
         x = layer.x_dev[start[rank]:start[rank + 1]].contiguous()
@@ -98,11 +101,11 @@ def _rank_worker(rank, sizes, port, q):
         dist.destroy_process_group()
 
 
-def _run_ranks(sizes):
+def _run_ranks(name, sizes):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_worker, args=(r, sizes, port, q)) for r in range(len(sizes))]
+    procs = [ctx.Process(target=_rank_worker, args=(r, name, sizes, port, q)) for r in range(len(sizes))]
     for p in procs:
         p.start()
     res = {}
@@ -127,13 +130,14 @@ def _run_ranks(sizes):
     return res
 
 
-@pytest.mark.parametrize("sizes", [(120, 77), (200, 0, 150, 300)])
-def test_ranks_as_processes_exchange_through_ipc(sizes):
+@pytest.mark.parametrize("name,sizes", [("e16", (120, 77)), ("e16", (200, 0, 150, 300)),
+                                        ("e256", (96, 96, 31, 1, 64, 0, 12, 100))])
+def test_ranks_as_processes_exchange_through_ipc(name, sizes):
     _require_shared_gpu()
     from token_dispatch_combine_b200 import MoEEPRank, ep_round_trip_one_gpu, moe_get_error
-    res = _run_ranks(sizes)
+    res = _run_ranks(name, sizes)
     R = len(sizes)
-    wl = _workload(sizes)
+    wl = _workload(name, sizes)
     layer = DeviceLayer(wl)
     start = np.concatenate([[0], np.cumsum(sizes)]).astype(int)
     xs = [layer.x_dev[start[r]:start[r + 1]].contiguous() for r in range(R)]
